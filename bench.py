@@ -1,0 +1,349 @@
+"""Benchmark of the Sol-Attn sparse attention forward (one JSON line on rank 0).
+
+A step is one call of the whole path -- pooling, routing, work ordering and
+the attention kernel -- on one seeded synthetic video-DiT-shaped input.  The
+default workload is Wan2.1-14B 720p attention (40 heads, L = 75600 on a
+21 x 45 x 80 latent grid, d = 128, blocks of 128) at beta = 1.04.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own
+independent call (its own seeded inputs): the heads of different calls do not
+interact, so there is no collective on the data path; timing is the max over
+ranks.  `--impl reference` times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/attention call and dense-equiv TFLOP/s at beta=1.04; % bf16 tensor peak"
+UNIT = "TFLOP/s (dense-equivalent)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+# ----------------------------------------------------------------------------- work accounting
+
+def executed_flops(sel: np.ndarray, L: int, B: int, d: int) -> dict:
+    """Algorithmic FLOPs of one call from the selection [b, H, N, N] (bool).
+
+    exact:  4 n_i n_j d for every selected pair (QK^T and PV);
+    approx: 2 n_i N d (token-to-pooled-key scores) + 2 n_i |U_i| d (pooled PV).
+    Padding, masked columns and skipped chunk columns are not counted.
+    """
+    N = sel.shape[-1]
+    n = np.full(N, B, dtype=np.float64)
+    n[-1] = L - (N - 1) * B
+    exact = 4.0 * d * np.einsum("bhij,i,j->", sel.astype(np.float64), n, n)
+    unsel = (~sel).sum(axis=-1).astype(np.float64)  # |U_i|, [b, H, N]
+    rows_with_approx = ((unsel > 0) * n[None, None, :]).sum()
+    approx = 2.0 * d * N * float(rows_with_approx) + 2.0 * d * float((unsel * n[None, None, :]).sum())
+    return {"exact": float(exact), "approx": float(approx), "total": float(exact + approx),
+            "selected_fraction": float(sel.mean())}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle timing (host)
+
+def oracle_sample_time(wl, beta: float, n_blocks: int = 2, seed: int = 0):
+    """Times the float64 oracle on one head's pooling + routing and `n_blocks`
+    query blocks of attention, and extrapolates to the whole call."""
+    from oracle import sol_attn as O
+    from video_diffusion_b200 import inputs as I
+    Q, K, V = I.make_qkv(wl.grid, 1, wl.d, wl.seed + seed, 1, wl.text_tokens, wl.dtype, "cpu")
+    Qh, Kh, Vh = (t[0, 0].double().numpy() for t in (Q, K, V))
+    t0 = time.perf_counter()
+    r = O.route_head(Qh, Kh, wl.block, wl.block, beta)
+    Vhat = O.pool_blocks(Vh, r["kgeom"], "sum")
+    t1 = time.perf_counter()
+    N = r["qgeom"].n
+    rng = np.random.default_rng(seed)
+    blocks = rng.choice(N, size=min(n_blocks, N), replace=False)
+    scale = 1.0 / math.sqrt(wl.d)
+    for i in blocks:
+        s0, n = int(r["qgeom"].starts[i]), int(r["qgeom"].counts[i])
+        O.attend_query_block(Qh[s0:s0 + n], Kh, Vh, r["kgeom"], r["Kbar"], Vhat, r["sel"][i], scale)
+    t2 = time.perf_counter()
+    per_head_prologue = t1 - t0
+    per_block = (t2 - t1) / len(blocks)
+    total = wl.batch * wl.heads * (per_head_prologue + per_block * N)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    sample = (f"1 head pooling+routing and {len(blocks)} of {N} query blocks, extrapolated to "
+              f"{wl.batch * wl.heads} heads x {N} blocks")
+    return total, cores, sample, float(r["sel"].mean())
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    for s in range(args.warmup + args.steps):
+        t, cores, sample, frac = oracle_sample_time(wl, args.beta, n_blocks=1, seed=s)
+        if s >= args.warmup:
+            times.append(t)
+    t = statistics.mean(times)
+    value = wl.dense_flops() / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, args):
+    return {"workload": wl.name, "beta": args.beta, "batch": wl.batch, "heads": wl.heads, "L": wl.L,
+            "d": wl.d, "block": wl.block, "parallelism": f"replicas x{args.gpus} (independent calls)",
+            "l2": "inputs 2.3 GB per step, larger than the 126 MB L2; no flush"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan-720p")
+    ap.add_argument("--beta", type=float, default=1.04)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from video_diffusion_b200 import inputs as I
+    wl = I.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    from video_diffusion_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if pg is None:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    Q, K, V = I.make_workload(wl, device=dev, seed_offset=rank)
+    out = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+
+    # selection statistics (same routing as the forward) for the FLOP count
+    counts, sel = api.stats(Q, K, args.beta, wl.block, with_mask=True)
+    work = executed_flops(sel.cpu().numpy(), wl.L, wl.block, wl.d)
+    del sel, counts
+
+    for _ in range(args.warmup):
+        api.forward(Q, K, V, args.beta, wl.block, out=out)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for s in range(args.steps):
+            api.forward_ex(Q, K, V, args.beta, wl.block, out=out, events=evs[s])
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = start.elapsed_time(end)
+    ms_step = max_over_ranks(total_ms / args.steps)
+    stage = {"pool": [], "route": [], "attention": []}
+    for e in evs:
+        stage["pool"].append(e[0].elapsed_time(e[1]))
+        stage["route"].append(e[1].elapsed_time(e[2]))
+        stage["attention"].append(e[2].elapsed_time(e[3]))
+    stage_ms = {k: statistics.mean(v) for k, v in stage.items()}
+    clock_summary = clocks.summary()
+
+    # in-house dense comparator: the same kernel with beta = -inf
+    dense_ms = None
+    if args.beta != -math.inf:
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        api.forward(Q, K, V, -math.inf, wl.block, out=out)
+        torch.cuda.synchronize()
+        d0.record(stream)
+        for _ in range(2):
+            api.forward(Q, K, V, -math.inf, wl.block, out=out)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = max_over_ranks(d0.elapsed_time(d1) / 2)
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+        hO = torch.empty_like(hQ).pin_memory()
+        dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 5))
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            dQ.copy_(hQ, non_blocking=True)
+            dK.copy_(hK, non_blocking=True)
+            dV.copy_(hV, non_blocking=True)
+            api.forward(dQ, dK, dV, args.beta, wl.block, out=out)
+            hO.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
+        e2e = {"value": world * wl.dense_flops() / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_call": e2e_ms,
+               "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+               "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n_e2e}
+        del hQ, hK, hV, hO, dQ, dK, dV
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, cores, sample, _ = oracle_sample_time(wl, args.beta, n_blocks=2)
+        cpu = {"value": wl.dense_flops() / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": sample, "extrapolated_s_per_call": t}
+
+    attn_ms = max_over_ranks(stage_ms["attention"])
+    achieved = work["total"] / (attn_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    value = world * wl.dense_flops() / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded smooth-field Q/K, V ~ N(0,1))",
+        "config": config_of(wl, args),
+        "ms_per_call": ms_step,
+        "selected_fraction": work["selected_fraction"],
+        "executed_tflop_per_call": work["total"] / 1e12,
+        "executed_tflops": work["total"] / (ms_step * 1e-3) / 1e12,
+        "pct_bf16_peak": 100.0 * work["total"] / (ms_step * 1e-3) / 1e12 / peak,
+        "stages_ms": stage_ms,
+        "dense_ms_per_call": dense_ms,
+        "speedup_vs_dense": (dense_ms / ms_step) if dense_ms else None,
+        "target_speedup": 1.0 / (work["selected_fraction"] + 0.15),
+        "roofline": {"kernel": "attn_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clock_summary,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,125 @@
+/*
+ * sol_attn.h -- C ABI of the B200 (sm_100a) Sol-Attn sparse attention forward.
+ *
+ * The operation (Sol-Attn visual explainer, mxino.github.io, "The complete idea
+ * in one pass", Eqs. 4, 5, 9, 10, 11): for every (batch, head)
+ *   1. pool:   Qbar_i = mean of the query rows of block i, Kbar_j = mean of the
+ *              key rows of block j, Vhat_j = sum of the value rows of block j
+ *              (blocks are contiguous runs of B tokens; the last may be partial,
+ *              with n_j < B tokens);
+ *   2. score:  s_ij = Qbar_i . Kbar_j / sqrt(d)                      (Eq. 4 legend)
+ *   3. route:  mu_i, sigma_i = mean and population std of row s_i.   (Eq. 5)
+ *              tau_i = mu_i + beta * sigma_i; S_i = { j : s_ij > tau_i } (Eq. 4)
+ *   4. attend: for every query token q of block i
+ *                D = sum_{j in U_i} n_j exp(q.Kbar_j/sqrt d) + sum_{j in S_i} sum_{k in j} exp(q.k/sqrt d)  (Eq. 9)
+ *                N = sum_{j in U_i} exp(q.Kbar_j/sqrt d) Vhat_j + sum_{j in S_i} sum_{k in j} exp(q.k/sqrt d) v_k (Eq. 10)
+ *              out = N / D, accumulated in one online-softmax pass.
+ * beta = -INFINITY selects every block (dense attention); beta = +INFINITY
+ * selects none (every block through its pooled key).  The 1/sqrt(d) logit
+ * scale is applied inside.  Rows are not masked (bidirectional attention).
+ *
+ * Conventions for every entry point
+ *   - Tensors are dense row-major [batch, heads, L, d] (d fastest), on the
+ *     current CUDA device, 16-byte aligned.  The caller owns them.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued on it; no call synchronises the host, except
+ *     sol_attn_device_status().
+ *   - Scratch memory (pooled tensors, the 1-bit selection mask, the work list;
+ *     about 4% of one input tensor) is taken with cudaMallocAsync on `stream`
+ *     and released with cudaFreeAsync on the same stream.
+ *   - Return value: SOL_OK or a negative sol_status.  Arguments are checked on
+ *     the host before anything is enqueued; on an argument error nothing is
+ *     enqueued.  Errors of kernels already enqueued surface at the caller's
+ *     next synchronisation, as usual in CUDA.
+ *   - Results are deterministic for a given input, shape and GPU.
+ */
+#ifndef SOL_ATTN_H
+#define SOL_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SOL_OK = 0,
+  SOL_ERR_INVALID_ARG = -1,     /* null/misaligned pointer, bad size, NaN beta */
+  SOL_ERR_UNSUPPORTED = -2,     /* valid but not built: see the support list below */
+  SOL_ERR_CUDA = -3,            /* a CUDA runtime call failed */
+  SOL_ERR_NO_MEMORY = -4,       /* scratch allocation failed */
+  SOL_ERR_DEVICE_TIMEOUT = -5   /* a kernel gave up on a bounded wait (see sol_attn_device_status) */
+} sol_status;
+
+typedef enum {
+  SOL_DTYPE_BF16 = 0,           /* bfloat16 inputs and output; fp32 accumulation */
+  SOL_DTYPE_F32 = 1             /* float32 inputs and output; fp32 arithmetic */
+} sol_dtype;
+
+/*
+ * Supported shapes: d in {64, 128}; Bq == Bk in {64, 128}; L >= 1;
+ * batch * heads >= 1; batch * heads * L * d < 2^31; beta not NaN.
+ * bf16 with d == 128 and B == 128 runs the tensor-core (tcgen05/TMEM/TMA)
+ * kernel; every other supported combination runs the CUDA-core kernel.
+ */
+
+/*
+ * Sparse attention forward, bf16.
+ *   q, k, v : const bf16*  [batch, heads, L, d], device
+ *   out     : bf16*        [batch, heads, L, d], device, written fully
+ *   Bq, Bk  : query / key block size in tokens (must be equal)
+ *   beta    : Eq. 4 knob; -INFINITY = dense, +INFINITY = all approximate
+ *   stream  : cudaStream_t
+ */
+int sol_attn_forward(const void* q, const void* k, const void* v, void* out,
+                     int batch, int heads, int L, int d, int Bq, int Bk,
+                     float beta, void* stream);
+
+/* Same operation on float32 tensors (fp32 arithmetic throughout). */
+int sol_attn_forward_f32(const float* q, const float* k, const float* v, float* out,
+                         int batch, int heads, int L, int d, int Bq, int Bk,
+                         float beta, void* stream);
+
+/*
+ * Selection statistics, computed by the same pooling and routing kernels as
+ * the forward (Eqs. 4-5).  No V is needed.
+ *   counts      : int32* [batch, heads, Nq] device; counts[.] = |S_i|
+ *   mask_or_null: uint32* [batch, heads, Nq, ceil(Nk/32)] device, or NULL;
+ *                 bit (j % 32) of word (j / 32) is 1 iff key block j is in S_i
+ *   dtype       : sol_dtype of q and k
+ * Nq = ceil(L/Bq), Nk = ceil(L/Bk).
+ */
+int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null,
+                   int batch, int heads, int L, int d, int Bq, int Bk,
+                   float beta, int dtype, void* stream);
+
+/*
+ * Extended forward for measurement.  Arguments as sol_attn_forward plus:
+ *   dtype  : sol_dtype of q, k, v, out
+ *   events : NULL, or 4 cudaEvent_t the library records on `stream`
+ *            before pooling, after pooling, after routing and after the
+ *            attention kernel (time each stage with cudaEventElapsedTime)
+ */
+int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, int dtype,
+                        int batch, int heads, int L, int d, int Bq, int Bk,
+                        float beta, void* const* events, void* stream);
+
+/*
+ * Reads and clears this device's status word, which a kernel sets when one of
+ * its bounded waits runs out (it then abandons its work and exits cleanly).
+ * Synchronises `stream` first.  Returns SOL_OK or SOL_ERR_DEVICE_TIMEOUT; if
+ * detail is not NULL it receives the raw word (0 = no error).
+ */
+int sol_attn_device_status(void* stream, int32_t* detail);
+
+/* Human-readable name of a sol_status value. */
+const char* sol_attn_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int sol_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_ATTN_H */

@@ -1,0 +1,80 @@
+"""Host checks of the C ABI: the library loads, exports every declared entry
+point, and rejects bad arguments before touching the GPU."""
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from video_diffusion_b200 import build, api
+    build.build()
+    return api.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "sol_attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sol_attn_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "sol_attn_forward" in names and "sol_attn_stats" in names
+    for n in names:
+        assert hasattr(L, n), n
+    from video_diffusion_b200 import api
+    assert set(api.EXPORTS) <= set(names)
+
+
+def test_status_strings_and_version(L):
+    from video_diffusion_b200 import api
+    assert api.status_string(0) == "SOL_OK"
+    assert api.status_string(-1) == "SOL_ERR_INVALID_ARG"
+    assert api.status_string(-5) == "SOL_ERR_DEVICE_TIMEOUT"
+    assert api.status_string(7) == "SOL_ERR_UNKNOWN"
+    assert api.version() == 100
+
+
+# Argument checks run on the host before any CUDA call, so fake device
+# addresses are never dereferenced.
+FAKE = 0x10000
+
+
+def call_fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, b=1, h=1, n=256, d=128, bq=128, bk=128, beta=1.0):
+    return L.sol_attn_forward(q, k, v, o, b, h, n, d, bq, bk, ctypes.c_float(beta), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(k=0), -1), (dict(v=0), -1), (dict(o=0), -1),
+    (dict(q=FAKE + 8), -1), (dict(o=FAKE + 2), -1),
+    (dict(b=0), -1), (dict(h=0), -1), (dict(n=0), -1), (dict(d=0), -1),
+    (dict(beta=float("nan")), -1),
+    (dict(d=96), -2), (dict(d=256), -2), (dict(bq=64, bk=128), -2), (dict(bq=32, bk=32), -2),
+    (dict(bq=256, bk=256), -2),
+])
+def test_forward_rejects_bad_arguments(L, kw, code):
+    assert call_fwd(L, **kw) == code
+
+
+def test_stats_and_ex_reject_bad_arguments(L):
+    f = ctypes.c_float
+    assert L.sol_attn_stats(FAKE, FAKE, None, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, None) == -1
+    assert L.sol_attn_stats(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 128, f(1.0), 9, None) == -1
+    assert L.sol_attn_stats(FAKE, FAKE, FAKE, None, 1, 1, 256, 100, 128, 128, f(1.0), 0, None) == -2
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 5, 1, 1, 256, 128, 128, 128, f(1.0), None, None) == -1
+    assert L.sol_attn_forward_f32(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 64, 64, f(math.nan), None) == -1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from video_diffusion_b200 import api
+    monkeypatch.setattr(api, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(api, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        api.lib()

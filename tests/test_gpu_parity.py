@@ -1,0 +1,171 @@
+"""GPU parity: the CUDA library (through its C ABI) against the float64 oracle.
+
+Selections must match the oracle's exactly except near-ties; outputs are
+compared element by element against the oracle run with the GPU's selection
+(which differs from its own only on near-ties).  Small cases are compared on
+every row; the full-size video workloads on every selection row and on a
+seeded sample of query blocks (first, last, max- and min-count, text blocks).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sol_attn as O
+from tests import parity_helpers as P
+from video_diffusion_b200 import api, build
+from video_diffusion_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+INF = math.inf
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    build.build()
+    api.lib()
+    yield
+    assert api.device_status() == 0
+
+
+def gpu_run(Q, K, V, block, beta):
+    out = torch.full_like(Q, float("nan"))
+    api.forward(Q, K, V, beta, block, out=out)
+    counts, sel = api.stats(Q, K, beta, block, with_mask=True)
+    torch.cuda.synchronize()
+    return out, counts.cpu().numpy(), sel.cpu().numpy()
+
+
+def check_case(Q, K, V, block, beta, sample_k=None, extra_blocks=(), seed=0, heads=None):
+    """Runs the GPU forward + stats and checks them against the oracle."""
+    b_, H, L, d = Q.shape
+    out, counts, sel = gpu_run(Q, K, V, block, beta)
+    rng = np.random.default_rng(seed)
+    stats = []
+    gpu_rows, ref_rows = [], []
+    for b in range(b_):
+        for h in range(H) if heads is None else heads:
+            r = O.route_head(P.head_np(Q, b, h), P.head_np(K, b, h), block, block, beta)
+            stats.append(P.compare_selection(r, sel[b, h], counts[b, h]))
+            N = r["qgeom"].n
+            if sample_k is None:
+                blocks = list(range(N))
+            else:
+                blocks = P.sample_blocks(N, counts[b, h], sample_k, rng, extra_blocks)
+            ref = P.oracle_rows(Q, K, V, b, h, block, beta, sel[b, h], blocks)
+            rows = P.rows_of(blocks, block, L)
+            ref_rows.append(ref[rows])
+            gpu_rows.append(out[b, h].double().cpu().numpy()[rows])
+    assert not torch.isnan(out).any(), "output rows left unwritten"
+    err = P.check_close(np.concatenate(gpu_rows), np.concatenate(ref_rows), Q.dtype, f"beta={beta}")
+    return err, stats
+
+
+# ------------------------------------------------------------------ small cases, every row
+
+@pytest.mark.parametrize("beta", [-INF, -1.0, 0.0, 0.5, 1.04, 2.0, INF])
+def test_bf16_ragged_full_rows(beta):
+    # L = 1000: 7 full blocks and a 104-token tail; several tiles per query block
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=7, batch=2, device="cuda")
+    check_case(Q, K, V, 128, beta)
+
+
+@pytest.mark.parametrize("beta", [-INF, 0.5, 1.04, INF])
+def test_tiny_fp32_workload(beta):
+    wl = I.WORKLOADS["tiny-fp32"]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    err, stats = check_case(Q, K, V, wl.block, beta)
+    assert err["rel_l2"] <= 1e-4
+
+
+@pytest.mark.parametrize("L", [1, 5, 127, 128, 129, 300])
+@pytest.mark.parametrize("beta", [-INF, 1.04, INF])
+def test_short_and_ragged_lengths(L, beta):
+    Q, K, V = I.make_iid(1, 3, L, 128, seed=L, dtype=torch.bfloat16, device="cuda")
+    check_case(Q, K, V, 128, beta)
+
+
+@pytest.mark.parametrize("d,block,dtype", [(128, 128, torch.float32), (64, 64, torch.bfloat16),
+                                           (64, 128, torch.bfloat16), (128, 64, torch.bfloat16),
+                                           (64, 64, torch.float32)])
+def test_other_shapes(d, block, dtype):
+    Q, K, V = I.make_qkv((3, 12, 20), heads=2, d=d, seed=11, dtype=dtype, device="cuda")  # L = 720
+    for beta in (-INF, 0.7, INF):
+        check_case(Q, K, V, block, beta)
+
+
+@pytest.mark.parametrize("beta", [-INF, 0.0, 1.04, INF])
+def test_identical_keys_per_block_equal_dense(beta):
+    """Keys constant inside each block: every beta gives dense attention."""
+    Q, K, V = I.make_iid(1, 2, 900, 128, seed=3, dtype=torch.float32, device="cuda")
+    N = -(-900 // 128)
+    Kb = torch.randn(1, 2, N, 128, device="cuda", generator=torch.Generator("cuda").manual_seed(5))
+    K = Kb.repeat_interleave(128, dim=2)[:, :, :900].contiguous()
+    Q, K, V = (t.to(torch.bfloat16).contiguous() for t in (Q, K, V))
+    out = api.forward(Q, K, V, beta, 128)
+    ref = O.dense_attention(Q.double().cpu().numpy(), K.double().cpu().numpy(), V.double().cpu().numpy())
+    P.check_close(out.double().cpu().numpy(), ref, torch.bfloat16, "identical keys")
+
+
+def test_deterministic_and_stream_ordered():
+    Q, K, V = I.make_qkv((6, 16, 16), heads=4, d=128, seed=9, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = api.forward(Q, K, V, 1.04)
+        b = api.forward(Q, K, V, 1.04)
+    s.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_invalid_arguments_raise():
+    Q, K, V = I.make_iid(1, 1, 256, 96, seed=1, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(api.SolAttnError):
+        api.forward(Q, K, V, 1.0)
+    Q, K, V = I.make_iid(1, 1, 256, 128, seed=1, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(api.SolAttnError):
+        api.forward(Q, K, V, float("nan"))
+
+
+# ------------------------------------------------------------------ workloads at full size
+
+@pytest.mark.parametrize("beta", [0.5, 1.04, 1.5])
+def test_image_dit(beta):
+    wl = I.WORKLOADS["image-dit"]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    check_case(Q, K, V, wl.block, beta, sample_k=3, heads=range(wl.heads), seed=1)
+
+
+@pytest.mark.parametrize("name,beta", [("wan-480p", 1.04),
+                                       ("wan-720p", -INF), ("wan-720p", 0.5), ("wan-720p", 1.04),
+                                       ("wan-720p", 1.5), ("wan-720p", 2.0),
+                                       ("hunyuan-720p", 1.04), ("hunyuan-720p", 1.5)])
+def test_video_workloads(name, beta):
+    wl = I.WORKLOADS[name]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    out, counts, sel = gpu_run(Q, K, V, wl.block, beta)
+    assert not torch.isnan(out).any()
+    rng = np.random.default_rng(2)
+    N = wl.n_blocks
+    text_blocks = ()
+    if wl.text_tokens:
+        first_text = (wl.L - wl.text_tokens) // wl.block
+        text_blocks = tuple(range(first_text, N))
+    sample_heads = [0, wl.heads // 2, wl.heads - 1]
+    gpu_rows, ref_rows = [], []
+    for h in range(wl.heads):
+        Qh, Kh = P.head_np(Q, 0, h), P.head_np(K, 0, h)
+        r = O.route_head(Qh, Kh, wl.block, wl.block, beta)
+        P.compare_selection(r, sel[0, h], counts[0, h])
+        if h in sample_heads:
+            k = 12 if beta != -INF else 4
+            blocks = P.sample_blocks(N, counts[0, h], k, rng, text_blocks)
+            ref = P.oracle_rows(Q, K, V, 0, h, wl.block, beta, sel[0, h], blocks)
+            rows = P.rows_of(blocks, wl.block, wl.L)
+            ref_rows.append(ref[rows])
+            gpu_rows.append(out[0, h].double().cpu().numpy()[rows])
+    P.check_close(np.concatenate(gpu_rows), np.concatenate(ref_rows), Q.dtype, f"{name} beta={beta}")
+    if beta == 1.04:
+        frac = sel.mean()
+        assert 0.05 < frac < 0.30, frac

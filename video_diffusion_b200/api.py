@@ -1,0 +1,166 @@
+"""Python binding of libsolattn (the C ABI in include/sol_attn.h).
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  If the
+compiled library is missing the first call raises; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
+_lib = None
+
+SOL_OK = 0
+STATUS = {0: "SOL_OK", -1: "SOL_ERR_INVALID_ARG", -2: "SOL_ERR_UNSUPPORTED", -3: "SOL_ERR_CUDA",
+          -4: "SOL_ERR_NO_MEMORY", -5: "SOL_ERR_DEVICE_TIMEOUT"}
+DTYPE_BF16, DTYPE_F32 = 0, 1
+
+EXPORTS = ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
+           "sol_attn_device_status", "sol_attn_status_string", "sol_attn_version")
+
+
+class SolAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libsolattn.so once; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with `python -m video_diffusion_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.sol_attn_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
+        L.sol_attn_forward_f32.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
+        L.sol_attn_forward_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, vp, vp]
+        L.sol_attn_stats.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
+        L.sol_attn_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+        L.sol_attn_status_string.argtypes = [i32]
+        L.sol_attn_status_string.restype = ctypes.c_char_p
+        L.sol_attn_version.argtypes = []
+        for name in ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
+                     "sol_attn_device_status", "sol_attn_version"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != SOL_OK:
+        raise SolAttnError(fn, rc)
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _shape(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor | None = None):
+    if q.dim() != 4:
+        raise ValueError("expected [batch, heads, L, d] tensors")
+    for t in (q, k) + ((v,) if v is not None else ()):
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, v must share shape, dtype and device")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    return q.shape
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, block: int = 128,
+            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Sol-Attn forward of [batch, heads, L, d] bf16 or fp32 tensors."""
+    b, h, L, d = _shape(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    fn = lib().sol_attn_forward if q.dtype == torch.bfloat16 else lib().sol_attn_forward_f32
+    _dtype_code(q)
+    rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b, h, L, d, block, block,
+            float(beta), _stream_handle(stream))
+    _check("sol_attn_forward", rc)
+    return out
+
+
+def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, stream=None) -> torch.Tensor:
+    """forward() that also records up to four torch.cuda.Event objects: before
+    pooling, after pooling, after routing, after the attention kernel."""
+    b, h, L, d = _shape(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    ev = None
+    if events is not None:
+        arr = (ctypes.c_void_p * 4)()
+        for i, e in enumerate(events):
+            arr[i] = int(e.cuda_event) if e is not None else 0
+        ev = ctypes.cast(arr, ctypes.c_void_p)
+    rc = lib().sol_attn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
+                                   b, h, L, d, block, block, float(beta), ev, _stream_handle(stream))
+    _check("sol_attn_forward_ex", rc)
+    return out
+
+
+def stats(q: torch.Tensor, k: torch.Tensor, beta: float, block: int = 128, with_mask: bool = False,
+          stream=None):
+    """Selected-block counts [batch, heads, Nq] (int32) and, if asked, the
+    selection as a bool tensor [batch, heads, Nq, Nk] unpacked from the
+    library's 1-bit mask."""
+    b, h, L, d = _shape(q, k)
+    N = -(-L // block)
+    W = -(-N // 32)
+    counts = torch.empty(b, h, N, dtype=torch.int32, device=q.device)
+    mask = torch.empty(b, h, N, W, dtype=torch.int32, device=q.device) if with_mask else None
+    rc = lib().sol_attn_stats(q.data_ptr(), k.data_ptr(), counts.data_ptr(),
+                              mask.data_ptr() if mask is not None else None, b, h, L, d, block, block,
+                              float(beta), _dtype_code(q), _stream_handle(stream))
+    _check("sol_attn_stats", rc)
+    if mask is None:
+        return counts
+    return counts, unpack_mask(mask, N)
+
+
+def unpack_mask(words: torch.Tensor, N: int) -> torch.Tensor:
+    """[..., W] int32 words -> [..., N] bool, bit j % 32 of word j // 32."""
+    shifts = torch.arange(32, device=words.device, dtype=torch.int64)
+    bits = (words.to(torch.int64).unsqueeze(-1) >> shifts) & 1
+    return bits.reshape(*words.shape[:-1], words.shape[-1] * 32)[..., :N].bool()
+
+
+def device_status(stream=None) -> int:
+    """Synchronises the stream, reads and clears the device status word."""
+    w = ctypes.c_int32(0)
+    rc = lib().sol_attn_device_status(_stream_handle(stream), ctypes.byref(w))
+    if rc not in (SOL_OK, -5):
+        _check("sol_attn_device_status", rc)
+    return int(w.value)
+
+
+def status_string(code: int) -> str:
+    return lib().sol_attn_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return int(lib().sol_attn_version())
+
+
+def n_blocks(L: int, block: int) -> int:
+    return -(-L // block)
+
+
+def beta_is_dense(beta: float) -> bool:
+    return beta == -math.inf

@@ -1,0 +1,200 @@
+// api.cu -- the C ABI of libsolattn (declared in include/sol_attn.h).
+//
+// Host-side work only: argument checks, scratch carving (one stream-ordered
+// allocation per call), and the launch sequence pool -> route -> order ->
+// attention on the caller's stream.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+
+#include "../../include/sol_attn.h"
+#include "common.cuh"
+
+namespace {
+
+using sol::Geometry;
+using sol::Scratch;
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_args(const void* q, const void* k, const void* v_or_dummy, const void* out_or_dummy, int batch,
+               int heads, int L, int d, int Bq, int Bk, float beta, Geometry* g) {
+  if (!q || !k || !v_or_dummy || !out_or_dummy) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v_or_dummy) || !aligned16(out_or_dummy))
+    return SOL_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || L < 1 || d < 1 || Bq < 1 || Bk < 1) return SOL_ERR_INVALID_ARG;
+  if (std::isnan(beta)) return SOL_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SOL_ERR_UNSUPPORTED;
+  if (Bq != Bk) return SOL_ERR_UNSUPPORTED;
+  if (Bq != 64 && Bq != 128) return SOL_ERR_UNSUPPORTED;
+  const int64_t bH = (int64_t)batch * heads;
+  if (bH > (1 << 24) || bH * (int64_t)L * d >= (int64_t(1) << 40)) return SOL_ERR_UNSUPPORTED;
+  const int B = Bq;
+  const int N = (L + B - 1) / B;
+  if (N > sol::kRouteMaxN) return SOL_ERR_UNSUPPORTED;
+  if (bH * N >= (int64_t(1) << 31)) return SOL_ERR_UNSUPPORTED;
+  g->bH = (int)bH;
+  g->L = L;
+  g->d = d;
+  g->B = B;
+  g->N = N;
+  g->W = (N + 31) / 32;
+  g->nchunk = (N + B - 1) / B;
+  g->n_last = L - (N - 1) * B;
+  g->nitems = (int)(bH * N);
+  return SOL_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Carves the scratch out of one allocation; returns its size when base is null.
+size_t carve(const Geometry& g, size_t op_elem, char* base, Scratch* s) {
+  const size_t pooled = (size_t)g.bH * g.N * g.d;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  s->qbar = reinterpret_cast<float*>(take(pooled * sizeof(float)));
+  s->kbar = reinterpret_cast<float*>(take(pooled * sizeof(float)));
+  s->kbar_op = take(pooled * op_elem);
+  s->vbar_op = take(pooled * op_elem);
+  s->mask = reinterpret_cast<uint32_t*>(take((size_t)g.nitems * g.W * sizeof(uint32_t)));
+  s->counts = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
+  s->tiles = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
+  s->order = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
+  s->work_counter = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
+  return off;
+}
+
+int beta_mode_of(float beta) { return std::isinf(beta) ? (beta < 0 ? -1 : 1) : 0; }
+
+uint64_t wait_limit_ns() {
+  // test hook: a shorter limit makes an expiring wait quick to observe
+  const char* e = std::getenv("SOL_ATTN_WAIT_LIMIT_NS");
+  if (e && *e) {
+    const unsigned long long v = std::strtoull(e, nullptr, 10);
+    if (v > 0) return v;
+  }
+  return kDefaultWaitLimitNs;
+}
+
+int record(void* const* events, int i, cudaStream_t st) {
+  if (!events || !events[i]) return SOL_OK;
+  return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+}
+
+int forward_impl(const void* q, const void* k, const void* v, void* out, int dtype, int batch, int heads, int L,
+                 int d, int Bq, int Bk, float beta, void* const* events, cudaStream_t st) {
+  if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
+  Geometry g;
+  int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
+  if (rc != SOL_OK) return rc;
+  const bool use_tc = dtype == SOL_DTYPE_BF16 && g.d == 128 && g.B == 128;
+  const int op_dtype = use_tc ? 0 : 1;  // operand type of K-bar / V-bar: bf16 for tensor cores
+  Scratch s;
+  const size_t bytes = carve(g, use_tc ? 2 : 4, nullptr, &s);
+  void* base = nullptr;
+  if (cudaMallocAsync(&base, bytes, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SOL_ERR_NO_MEMORY;
+  }
+  carve(g, use_tc ? 2 : 4, static_cast<char*>(base), &s);
+  cudaError_t e = cudaSuccess;
+  const int in_dtype = dtype == SOL_DTYPE_BF16 ? 0 : 1;
+  if ((rc = record(events, 0, st)) != SOL_OK) goto done;
+  e = sol::launch_pool(in_dtype, op_dtype, q, k, v, g, s, st);
+  if (e != cudaSuccess) goto done;
+  if ((rc = record(events, 1, st)) != SOL_OK) goto done;
+  e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, st);
+  if (e != cudaSuccess) goto done;
+  e = sol::launch_order(g, s, st);
+  if (e != cudaSuccess) goto done;
+  if ((rc = record(events, 2, st)) != SOL_OK) goto done;
+  if (use_tc) {
+    e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) goto done;
+    e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns());
+  } else {
+    e = sol::launch_attn_simt(in_dtype, q, k, v, out, g, s, st);
+  }
+  if (e != cudaSuccess) goto done;
+  rc = record(events, 3, st);
+done:
+  cudaFreeAsync(base, st);
+  if (e != cudaSuccess) return SOL_ERR_CUDA;
+  return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sol_attn_forward(const void* q, const void* k, const void* v, void* out, int batch, int heads, int L, int d,
+                     int Bq, int Bk, float beta, void* stream) {
+  return forward_impl(q, k, v, out, SOL_DTYPE_BF16, batch, heads, L, d, Bq, Bk, beta, nullptr,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_forward_f32(const float* q, const float* k, const float* v, float* out, int batch, int heads, int L,
+                         int d, int Bq, int Bk, float beta, void* stream) {
+  return forward_impl(q, k, v, out, SOL_DTYPE_F32, batch, heads, L, d, Bq, Bk, beta, nullptr,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, int dtype, int batch, int heads,
+                        int L, int d, int Bq, int Bk, float beta, void* const* events, void* stream) {
+  return forward_impl(q, k, v, out, dtype, batch, heads, L, d, Bq, Bk, beta, events,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int batch, int heads,
+                   int L, int d, int Bq, int Bk, float beta, int dtype, void* stream) {
+  if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
+  if (!counts) return SOL_ERR_INVALID_ARG;
+  Geometry g;
+  int rc = check_args(q, k, q, q, batch, heads, L, d, Bq, Bk, beta, &g);
+  if (rc != SOL_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch s;
+  const size_t bytes = carve(g, 4, nullptr, &s);
+  void* base = nullptr;
+  if (cudaMallocAsync(&base, bytes, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SOL_ERR_NO_MEMORY;
+  }
+  carve(g, 4, static_cast<char*>(base), &s);
+  s.counts = counts;
+  if (mask_or_null) s.mask = mask_or_null;
+  s.kbar_op = nullptr;  // routing needs the fp32 pooled vectors only
+  cudaError_t e = sol::launch_pool(dtype == SOL_DTYPE_BF16 ? 0 : 1, 1, q, k, nullptr, g, s, st);
+  if (e == cudaSuccess) e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, st);
+  cudaFreeAsync(base, st);
+  return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+}
+
+int sol_attn_device_status(void* stream, int32_t* detail) {
+  int32_t w = 0;
+  if (sol::read_device_status(static_cast<cudaStream_t>(stream), &w) != cudaSuccess) return SOL_ERR_CUDA;
+  if (detail) *detail = w;
+  return w == 0 ? SOL_OK : SOL_ERR_DEVICE_TIMEOUT;
+}
+
+const char* sol_attn_status_string(int status) {
+  switch (status) {
+    case SOL_OK: return "SOL_OK";
+    case SOL_ERR_INVALID_ARG: return "SOL_ERR_INVALID_ARG";
+    case SOL_ERR_UNSUPPORTED: return "SOL_ERR_UNSUPPORTED";
+    case SOL_ERR_CUDA: return "SOL_ERR_CUDA";
+    case SOL_ERR_NO_MEMORY: return "SOL_ERR_NO_MEMORY";
+    case SOL_ERR_DEVICE_TIMEOUT: return "SOL_ERR_DEVICE_TIMEOUT";
+    default: return "SOL_ERR_UNKNOWN";
+  }
+}
+
+int sol_attn_version(void) { return 100; }
+
+}  // extern "C"

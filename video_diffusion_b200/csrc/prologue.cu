@@ -1,0 +1,321 @@
+// prologue.cu -- block pooling, proxy scores, Eq. 4 routing and the work order.
+//
+// Sol-Attn visual explainer (mxino.github.io):
+//   "Pool Q, K and V into blocks" -> pool_kernel: Q-bar_i, K-bar_j are block
+//     means, V-hat_j the block sum (stored divided by n_j, with log n_j added to
+//     the pooled logit by the attention kernel: n_j e^a V-hat_j/n_j / (n_j e^a)).
+//   Eq. 4 / Eq. 5 -> route_kernel: the proxy row s_i = Q-bar_i K-bar^T / sqrt(d)
+//     is formed on chip (shared memory), its mean and population standard
+//     deviation give tau_i = mu_i + beta sigma_i, and S_i = {j : s_ij > tau_i}
+//     leaves as one bit per pair.  No N x N score map reaches global memory.
+// All reductions run in a fixed order, so results are deterministic.
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace sol {
+namespace {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+constexpr int kPoolThreads = 256;
+
+// Sum of the rows [r0, r0 + n) of X ([rows, D] slice of one head), one 16-byte
+// column group per thread: thread (cg, rl) adds rows rl, rl + R, ... of its
+// group; the R partial sums are then added in shared memory in fixed order.
+template <typename T, int D>
+__device__ void block_column_sums(const T* __restrict__ X, int n, float* __restrict__ red, float* __restrict__ out) {
+  constexpr int VEC = 16 / sizeof(T);   // elements per 16-byte load
+  constexpr int G = D / VEC;            // column groups per row
+  constexpr int R = kPoolThreads / G;   // row lanes
+  const int tid = threadIdx.x;
+  const int cg = tid % G, rl = tid / G;
+  float acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  // Issue several independent 16-byte loads before adding them.
+  constexpr int U = 4;
+  int r = rl;
+  for (; r + (U - 1) * R < n; r += U * R) {
+    uint4 raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      raw[u] = __ldcs(reinterpret_cast<const uint4*>(X + (size_t)(r + u * R) * D) + cg);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const T* e8 = reinterpret_cast<const T*>(&raw[u]);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] += to_f(e8[e]);
+    }
+  }
+  for (; r < n; r += R) {
+    uint4 raw = __ldcs(reinterpret_cast<const uint4*>(X + (size_t)r * D) + cg);
+    const T* e8 = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] += to_f(e8[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) red[rl * D + cg * VEC + e] = acc[e];
+  __syncthreads();
+  for (int c = tid; c < D; c += kPoolThreads) {
+    float s = 0.f;
+    for (int q = 0; q < R; ++q) s += red[q * D + c];
+    out[c] = s;
+  }
+  __syncthreads();
+}
+
+// grid (N, bH).  Q-bar (fp32), K-bar (fp32 and operand type), V-hat/n (operand type).
+template <typename T, typename Op, int D>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                            const T* __restrict__ v, int L, int B, int N,
+                                                            float* __restrict__ qbar, float* __restrict__ kbar,
+                                                            Op* __restrict__ kbar_op, Op* __restrict__ vbar_op) {
+  constexpr int VEC = 16 / sizeof(T);
+  constexpr int R = kPoolThreads / (D / VEC);
+  __shared__ float red[R * D];
+  __shared__ float sums[D];
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int r0 = blk * B;
+  const int n = min(B, L - r0);
+  const float inv_n = 1.0f / (float)n;
+  const size_t head = (size_t)bh * L * D + (size_t)r0 * D;
+  const size_t prow = ((size_t)bh * N + blk) * D;
+
+  block_column_sums<T, D>(q + head, n, red, sums);
+  for (int c = threadIdx.x; c < D; c += kPoolThreads) qbar[prow + c] = sums[c] * inv_n;
+  block_column_sums<T, D>(k + head, n, red, sums);
+  for (int c = threadIdx.x; c < D; c += kPoolThreads) {
+    float m = sums[c] * inv_n;
+    kbar[prow + c] = m;
+    if (kbar_op) kbar_op[prow + c] = from_f<Op>(m);
+  }
+  if (v != nullptr) {
+    block_column_sums<T, D>(v + head, n, red, sums);
+    for (int c = threadIdx.x; c < D; c += kPoolThreads) vbar_op[prow + c] = from_f<Op>(sums[c] * inv_n);
+  }
+}
+
+constexpr int kRouteThreads = 256;
+constexpr int kRouteKC = 32;  // pooled keys staged in shared memory at a time
+
+// grid (ceil(N / QB), bH), 256 threads.  Each warp owns one query block of
+// the group for the row statistics; the score pass pairs warp w with query
+// block w and lane l with key l of the staged chunk.
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __restrict__ qbar,
+                                                              const float* __restrict__ kbar, int N, int W,
+                                                              int B, int nchunk, int QB, float scale, float beta,
+                                                              int beta_mode, int correction,
+                                                              uint32_t* __restrict__ mask,
+                                                              int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ tiles) {
+  extern __shared__ float sm[];
+  float* qs = sm;                          // [QB][D]
+  float* ks = qs + QB * D;                 // [KC][D + 1]
+  float* srow = ks + kRouteKC * (D + 1);   // [QB][N]
+  const int bh = blockIdx.y;
+  const int i0 = blockIdx.x * QB;
+  const int nq = min(QB, N - i0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* qb = qbar + ((size_t)bh * N + i0) * D;
+  const float* kb = kbar + (size_t)bh * N * D;
+
+  for (int e = tid; e < nq * D; e += kRouteThreads) qs[e] = qb[e];
+  for (int j0 = 0; j0 < N; j0 += kRouteKC) {
+    const int nk = min(kRouteKC, N - j0);
+    __syncthreads();
+    for (int e = tid; e < nk * D; e += kRouteThreads) {
+      int jj = e / D, c = e % D;
+      ks[jj * (D + 1) + c] = kb[(size_t)(j0 + jj) * D + c];
+    }
+    __syncthreads();
+    for (int qi = warp; qi < nq; qi += kRouteThreads / 32) {
+      if (lane < nk) {
+        const float* qv = qs + qi * D;
+        const float* kv = ks + lane * (D + 1);
+        float s = 0.f;
+#pragma unroll 16
+        for (int c = 0; c < D; ++c) s = fmaf(qv[c], kv[c], s);
+        srow[(size_t)qi * N + j0 + lane] = s * scale;
+      }
+    }
+  }
+  __syncthreads();
+
+  for (int qi = warp; qi < nq; qi += kRouteThreads / 32) {
+    const float* s = srow + (size_t)qi * N;
+    // mean and population variance, two passes, lane-strided then a fixed tree
+    float a = 0.f;
+    for (int j = lane; j < N; j += 32) a += s[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    const float mu = a / (float)N;
+    float v = 0.f;
+    for (int j = lane; j < N; j += 32) {
+      float t = s[j] - mu;
+      v = fmaf(t, t, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const float sigma = sqrtf(v / (float)N);
+    float tau;
+    if (beta_mode < 0) tau = -INFINITY;
+    else if (beta_mode > 0) tau = INFINITY;
+    else tau = fmaf(beta, sigma, mu);
+
+    const size_t item = (size_t)bh * N + i0 + qi;
+    uint32_t* mrow = mask + item * W;
+    int cnt = 0;
+    for (int w = lane; w < W; w += 32) {
+      uint32_t bits = 0;
+      const int jb = w * 32;
+      const int nb = min(32, N - jb);
+      for (int b = 0; b < nb; ++b) bits |= (s[jb + b] > tau ? 1u : 0u) << b;
+      mrow[w] = bits;
+      cnt += __popc(bits);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    // pooled-key chunks holding at least one unselected block
+    int used = 0;
+    if (correction) {
+      const int wpc = B / 32;  // mask words per chunk
+      for (int c = lane; c < nchunk; c += 32) {
+        bool any = false;
+        for (int q = 0; q < wpc; ++q) {
+          const int w = c * wpc + q;
+          if (w >= W) break;
+          const int jb = w * 32;
+          const int nb = min(32, N - jb);
+          const uint32_t valid = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+          // recompute from scores: the words above may belong to other lanes
+          uint32_t bits = 0;
+          for (int b = 0; b < nb; ++b) bits |= (s[jb + b] > tau ? 1u : 0u) << b;
+          any |= ((~bits) & valid) != 0u;
+        }
+        used += any ? 1 : 0;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) used += __shfl_xor_sync(0xffffffffu, used, o);
+    }
+    if (lane == 0) {
+      counts[item] = cnt;
+      tiles[item] = cnt + used;
+    }
+  }
+}
+
+// One CTA per head: bitonic sort of the head's work items by (tiles desc,
+// index asc); writes order[bh * N + rank] = bh * N + i.
+__global__ void __launch_bounds__(1024) order_kernel(const int32_t* __restrict__ tiles, int N, int P,
+                                                     int32_t* __restrict__ order) {
+  extern __shared__ unsigned long long keys[];
+  const int bh = blockIdx.x;
+  for (int e = threadIdx.x; e < P; e += blockDim.x) {
+    unsigned long long key;
+    if (e < N) {
+      const uint32_t t = (uint32_t)tiles[(size_t)bh * N + e];
+      key = ((unsigned long long)(0x7fffffffu - t) << 32) | (uint32_t)e;
+    } else {
+      key = ~0ull;
+    }
+    keys[e] = key;
+  }
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int e = threadIdx.x; e < P; e += blockDim.x) {
+        const int partner = e ^ stride;
+        if (partner > e) {
+          const bool up = (e & size) == 0;
+          unsigned long long a = keys[e], b = keys[partner];
+          if ((a > b) == up) {
+            keys[e] = b;
+            keys[partner] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int e = threadIdx.x; e < N; e += blockDim.x)
+    order[(size_t)bh * N + e] = bh * N + (int)(uint32_t)(keys[e] & 0xffffffffu);
+}
+
+__global__ void identity_order_kernel(int32_t* order, int n) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) order[e] = e;
+}
+
+template <typename T, typename Op>
+cudaError_t pool_dispatch(const void* q, const void* k, const void* v, const Geometry& g, const Scratch& s,
+                          cudaStream_t st) {
+  dim3 grid(g.N, g.bH);
+  if (g.d == 128)
+    pool_kernel<T, Op, 128><<<grid, kPoolThreads, 0, st>>>(
+        (const T*)q, (const T*)k, (const T*)v, g.L, g.B, g.N, s.qbar, s.kbar, (Op*)s.kbar_op, (Op*)s.vbar_op);
+  else
+    pool_kernel<T, Op, 64><<<grid, kPoolThreads, 0, st>>>(
+        (const T*)q, (const T*)k, (const T*)v, g.L, g.B, g.N, s.qbar, s.kbar, (Op*)s.kbar_op, (Op*)s.vbar_op);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// in_dtype / op_dtype: 0 = bf16, 1 = fp32.
+cudaError_t launch_pool(int in_dtype, int op_dtype, const void* q, const void* k, const void* v,
+                        const Geometry& g, const Scratch& s, cudaStream_t st) {
+  if (in_dtype == 0 && op_dtype == 0) return pool_dispatch<__nv_bfloat16, __nv_bfloat16>(q, k, v, g, s, st);
+  if (in_dtype == 0 && op_dtype == 1) return pool_dispatch<__nv_bfloat16, float>(q, k, v, g, s, st);
+  if (in_dtype == 1 && op_dtype == 1) return pool_dispatch<float, float>(q, k, v, g, s, st);
+  return pool_dispatch<float, __nv_bfloat16>(q, k, v, g, s, st);
+}
+
+static int route_qb(int N) {
+  // query blocks per CTA, bounded by the shared memory their score rows take
+  int qb = 8;
+  while (qb > 1 && (size_t)qb * N * sizeof(float) > 160u * 1024u) qb >>= 1;
+  return qb;
+}
+
+cudaError_t launch_route(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
+                         cudaStream_t st) {
+  const int QB = route_qb(g.N);
+  const size_t smem = (size_t)(QB * g.d + kRouteKC * (g.d + 1) + (size_t)QB * g.N) * sizeof(float);
+  dim3 grid((g.N + QB - 1) / QB, g.bH);
+  const float scale = 1.0f / sqrtf((float)g.d);
+  cudaError_t e;
+  if (g.d == 128) {
+    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<128><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, g.N, g.W, g.B, g.nchunk, QB, scale, beta,
+                                                         beta_mode, correction, s.mask, s.counts, s.tiles);
+  } else {
+    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<64><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, g.N, g.W, g.B, g.nchunk, QB, scale, beta,
+                                                        beta_mode, correction, s.mask, s.counts, s.tiles);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st) {
+  if (g.N > kOrderMaxN) {
+    identity_order_kernel<<<148, 256, 0, st>>>(s.order, g.nitems);
+    return cudaGetLastError();
+  }
+  int P = 1;
+  while (P < g.N) P <<= 1;
+  const size_t smem = (size_t)P * sizeof(unsigned long long);
+  cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  order_kernel<<<g.bH, 1024, smem, st>>>(s.tiles, g.N, P, s.order);
+  return cudaGetLastError();
+}
+
+}  // namespace sol
