@@ -188,6 +188,40 @@ def config_of(wl, args):
             "l2": "inputs 2.3 GB per step, larger than the 126 MB L2; no flush"}
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_info():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def setup_dist(world: int, backend: str, device=None):
+    """Process group for N > 1 (short timeout so a missing rank ends in an
+    error, not a wait); None when running alone."""
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    kw = {"device_id": device} if backend == "nccl" else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def reduce_max(x: float, pg, device) -> float:
+    """Max of x over ranks (the job's time is its slowest rank's)."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world: int, flops_per_call: float, ms_per_call: float) -> float:
+    """Whole-job dense-equivalent TFLOP/s: every rank runs one call per step."""
+    return world * flops_per_call / (ms_per_call * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
@@ -211,28 +245,17 @@ def main():
 
     from video_diffusion_b200 import api
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_info()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
+    pg = setup_dist(world, "nccl", dev)
 
     def barrier():
         if pg is not None:
             pg.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if pg is None:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, pg, dev)
 
     peaks = load_peaks()
     Q, K, V = I.make_workload(wl, device=dev, seed_offset=rank)
@@ -249,6 +272,9 @@ def main():
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for row in evs:  # torch creates the CUDA event on first record; the library then re-records it
+        for e in row:
+            e.record(stream)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -302,7 +328,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
-        e2e = {"value": world * wl.dense_flops() / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_call": e2e_ms,
+        e2e = {"value": aggregate_value(world, wl.dense_flops(), e2e_ms), "unit": UNIT, "ms_per_call": e2e_ms,
                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n_e2e}
         del hQ, hK, hV, hO, dQ, dK, dV
@@ -316,7 +342,7 @@ def main():
     attn_ms = max_over_ranks(stage_ms["attention"])
     achieved = work["total"] / (attn_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    value = world * wl.dense_flops() / (ms_step * 1e-3) / 1e12
+    value = aggregate_value(world, wl.dense_flops(), ms_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

@@ -99,7 +99,8 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, bloc
 
 def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, stream=None) -> torch.Tensor:
     """forward() that also records up to four torch.cuda.Event objects: before
-    pooling, after pooling, after routing, after the attention kernel."""
+    pooling, after pooling, after routing, after the attention kernel.  The
+    events must exist already (torch creates them on their first record())."""
     b, h, L, d = _shape(q, k, v)
     if out is None:
         out = torch.empty_like(q)
@@ -108,6 +109,8 @@ def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, st
         arr = (ctypes.c_void_p * 4)()
         for i, e in enumerate(events):
             arr[i] = int(e.cuda_event) if e is not None else 0
+            if e is not None and arr[i] is None:
+                raise ValueError("event not created yet: record it once before passing it")
         ev = ctypes.cast(arr, ctypes.c_void_p)
     rc = lib().sol_attn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
                                    b, h, L, d, block, block, float(beta), ev, _stream_handle(stream))
