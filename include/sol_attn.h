@@ -112,6 +112,27 @@ int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, 
  */
 int sol_attn_device_status(void* stream, int32_t* detail);
 
+/*
+ * Forward without any memory allocation, for callers that may not allocate
+ * device memory (plugin hosts that own all device memory, serving loops that
+ * reserve everything up front and treat an allocation as a failure).  The
+ * paper has no counterpart; the computation is that of sol_attn_forward, with
+ * the same arguments, kernels and results.
+ *   - Scratch comes from a fixed 48 MiB device array inside the library,
+ *     present on every GPU that loads it until the process exits.  A call
+ *     whose scratch would not fit returns SOL_ERR_NO_MEMORY before enqueueing
+ *     anything (the Wan2.1 720p and HunyuanVideo 720p calls fit).
+ *   - The first call on a device looks up the array's device address (a
+ *     cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the array, and it keeps the previous call's
+ *     contents (the call resets what must start at zero).  Calls that overlap
+ *     on the GPU -- e.g. on two streams without ordering between them -- race
+ *     on it: keep them ordered.
+ */
+int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out,
+                             int batch, int heads, int L, int d, int Bq, int Bk,
+                             float beta, void* stream);
+
 /* Human-readable name of a sol_status value. */
 const char* sol_attn_status_string(int status);
 

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <mutex>
 
 #include "../../include/sol_attn.h"
 #include "common.cuh"
@@ -198,3 +199,75 @@ const char* sol_attn_status_string(int status) {
 int sol_attn_version(void) { return 100; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------- forward without allocation
+//
+// Some callers cannot let a library allocate device memory: runtimes that load
+// this code as a plugin and hand out every byte of device memory themselves,
+// and serving loops that reserve all memory up front and treat any further
+// allocation (which can block, fail under fragmentation, or take memory meant
+// for activations) as an error.  sol_attn_forward_noalloc serves them with the
+// same kernels as sol_attn_forward, taking its scratch from the fixed array
+// below instead of cudaMallocAsync.
+
+namespace {
+
+// Fixed scratch, reserved on every GPU that loads this library until the
+// process exits.  48 MiB holds the scratch of the Wan2.1 720p call (40 heads,
+// L = 75600: about 38 MiB) and of the HunyuanVideo 720p call.
+constexpr size_t kNoAllocScratchBytes = size_t(48) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name only stands in for the symbol; the address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SOL_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SOL_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return SOL_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SOL_OK;
+}
+
+}  // namespace
+
+extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int batch,
+                                        int heads, int L, int d, int Bq, int Bk, float beta, void* stream) {
+  Geometry g;
+  int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
+  if (rc != SOL_OK) return rc;
+  const bool use_tc = g.d == 128 && g.B == 128;
+  const int op_dtype = use_tc ? 0 : 1;
+  Scratch s;
+  const size_t bytes = carve(g, use_tc ? 2 : 4, nullptr, &s);
+  if (bytes > kNoAllocScratchBytes) return SOL_ERR_NO_MEMORY;  // call too large for the fixed scratch
+  void* base = nullptr;
+  if ((rc = noalloc_scratch(&base)) != SOL_OK) return rc;
+  carve(g, use_tc ? 2 : 4, static_cast<char*>(base), &s);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Everything the kernels read is rewritten by this call except the work
+  // counter, which must start at zero.
+  cudaError_t e = sol::launch_pool(0, op_dtype, q, k, v, g, s, st);
+  if (e == cudaSuccess) e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, st);
+  if (e == cudaSuccess) e = sol::launch_order(g, s, st);
+  if (use_tc) {
+    if (e == cudaSuccess) e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
+    if (e == cudaSuccess) e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns());
+  } else if (e == cudaSuccess) {
+    e = sol::launch_attn_simt(0, q, k, v, out, g, s, st);
+  }
+  return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+}
