@@ -13,13 +13,18 @@
 //     past the block's n_j tokens, and O += P V_j (Eqs. 9, 10 "Exact" terms).
 //     Only selected K/V tiles are ever loaded.
 //
-// Persistent CTAs, one per SM, 192 threads:
-//   warp 0      TMA producer: Q tile, then K/V (or K-bar/V-bar) tiles in a
-//               3-stage K ring and a 2-stage V ring; fetches work items
-//   warp 1      TMEM owner and single-thread tcgen05.mma issuer
-//   warps 2..5  softmax: one query row per thread (TMEM lane), P to TMEM,
-//               lazy O rescaling, epilogue
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
+// Persistent CTAs, one per SM, 320 threads:
+//   warp 0      TMA producer: fetches work items, loads Q tiles (2 buffers)
+//               and K/V (or K-bar/V-bar) tiles (2-stage K and V rings)
+//   warp 1      TMEM owner and tcgen05.mma issuer (one elected lane)
+//   warps 2..9  softmax, two column halves: half h owns the 64 keys
+//               [64h, 64h + 64) of every tile, one query row per thread (its
+//               warp's TMEM lane quadrant).  Each half keeps its own running
+//               max, row sum and fp32 accumulator O_h = sum P_h V_h, so the
+//               halves never wait for each other inside the key loop; the two
+//               partial softmax states of a row are merged once per item.
+// TMEM columns: S [0,128), O_0 [128,256), O_1 [256,384), P [384,512) as two
+// buffers of 64 columns, each holding half 0's then half 1's 64 bf16 pairs.
 // Every mbarrier wait is bounded; on expiry the CTA abandons its work, waits
 // for its own copies and MMAs, frees TMEM and records the failing wait in the
 // device status word.
@@ -36,18 +41,25 @@ __device__ int g_sol_status;  // 0 = ok; else 0x1000 | wait id (first expiry)
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int KST = 3, VST = 2;
-constexpr int NTHREADS = 192;
+constexpr int QST = 2, KST = 2, VST = 2;
+constexpr int NTHREADS = 320;
+constexpr int SOFTMAX_WARPS = 8;
 constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB, two 64-column swizzled halves
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = TILE_BYTES;
+constexpr uint32_t OFF_K = OFF_Q + QST * TILE_BYTES;
 constexpr uint32_t OFF_V = OFF_K + KST * TILE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_V + VST * TILE_BYTES;  // 192 KB
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barriers + alignment slack
+constexpr uint32_t BAR_AREA = 8192;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA + 1024;  // + alignment slack
 
-constexpr uint32_t TM_S = 0, TM_O = 256, TM_P = 384;
+constexpr uint32_t TM_S = 0, TM_O = 128, TM_P = 384;  // O_h at TM_O + 128 h
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+// One column pair in POLY_PAIR_PERIOD takes the FMA-pipe polynomial exp2
+// instead of the MUFU ex2 unit (16 of a thread's 64 columns per tile): per
+// tile the MUFU unit, not the FMA pipe, is the tighter of the two.
+constexpr int POLY_PAIR_PERIOD = 4;
 
 struct Params {
   int bH, L, N, W, nchunk, nitems, n_last;
@@ -63,19 +75,23 @@ struct Params {
 };
 
 struct Bars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[QST], q_empty[QST];
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];  // per P buffer: the PV MMA that read it has finished
+  uint64_t s_full, s_free;
+  uint64_t p_full[2][2];  // [P buffer][column half]
+  uint64_t pv_done[2];    // per P buffer: both PV MMAs that read it have finished
   uint64_t o_full, o_free;
   uint64_t item_full[2], item_empty[2];
+  uint64_t xstate;        // softmax-state exchange between the halves at the end of an item
   uint64_t teardown;
   int item_slot[2];
   uint32_t tmem_base;
   int abort_flag;
+  float xm[2][2][BM];     // [item parity][column half][row] running max (log2 units)
+  float xl[2][2][BM];     // [item parity][column half][row] row sum
 };
+static_assert(sizeof(Bars) <= BAR_AREA, "barrier area");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
 // unselected block, then the selected blocks in increasing order.
@@ -117,33 +133,44 @@ struct TileIter {
   }
 };
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars& B_, uint64_t lim, int id) {
-  return mbar_wait(bar, parity, &B_.abort_flag, &g_sol_status, 0x1000 | id, lim);
-}
-// All 32 lanes wait; the outcome is made warp-uniform so that the warp-wide
-// tcgen05.ld/st that follow are never reached by part of a warp.
-__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Bars& B_, uint64_t lim, int id) {
-  const bool ok = wait_bar(bar, parity, B_, lim, id);
+// All 32 lanes wait; the outcome is made warp-uniform so that warp-wide
+// instructions that follow are never reached by part of a warp.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Bars& B_, uint64_t lim, int id) {
+  const bool ok = mbar_wait(bar, parity, &B_.abort_flag, &g_sol_status, 0x1000 | id, lim);
   return __all_sync(0xffffffffu, ok);
 }
 
-// ------------------------------------------------------------------ softmax helpers
-// u_c = s_c * scale_log2 + bias_c for valid columns, -inf otherwise; returns max.
-template <bool FULL>
-__device__ __forceinline__ float tile_logits(float (&x)[128], float sl2, float bias, const uint32_t (&vm)[4],
-                                             int sc, float sc_delta) {
-  float rmax = -INFINITY;
+// 2^x for x <= 8 on the FMA pipe: x = j + f with j = round(x), f in [-1/2, 1/2];
+// 2^f from a cubic fitted here to 2^f on [-1/2, 1/2] (least squares with
+// Lawson reweighting toward minimax relative error, max 7.5e-5), then j is
+// added to the exponent field.  Inputs below -125 (where the exponent field
+// would underflow) give exactly 0, as does -inf.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 xc = make_float2(fmaxf(x.x, -125.0f), fmaxf(x.y, -125.0f));
+  const float shifter = 12582912.0f;  // 1.5 * 2^23: xc + shifter rounds xc to an integer in the low bits
+  const float2 t = add2(xc, make_float2(shifter, shifter));
+  const float2 j = add2(t, make_float2(-shifter, -shifter));
+  const float2 f = add2(xc, make_float2(-j.x, -j.y));
+  float2 p = fma2(make_float2(0.05517118f, 0.05517118f), f, make_float2(0.24261113f, 0.24261113f));
+  p = fma2(p, f, make_float2(0.69326109f, 0.69326109f));
+  p = fma2(p, f, make_float2(0.99992806f, 0.99992806f));
+  // the low bits of t hold j; shifting them into the exponent field adds j to p's exponent
+  const float r0 = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
+  return make_float2(x.x < -125.0f ? 0.0f : r0, x.y < -125.0f ? 0.0f : r1);
+}
+
+// Max of 64 values with three-input max instructions.
+__device__ __forceinline__ float tree_max64(const float (&x)[64]) {
+  float a[22];
 #pragma unroll
-  for (int c = 0; c < 128; ++c) {
-    float u = fmaf(x[c], sl2, bias);
-    if (!FULL) {
-      if (c == sc) u += sc_delta;
-      if (!((vm[c >> 5] >> (c & 31)) & 1u)) u = -INFINITY;
-    }
-    x[c] = u;
-    rmax = fmaxf(rmax, u);
-  }
-  return rmax;
+  for (int i = 0; i < 21; ++i) a[i] = max3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+  a[21] = x[63];
+  float b[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) b[i] = max3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[7] = a[21];
+  return max3(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -157,20 +184,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint64_t lim = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.q_empty, 1);
+    for (int s = 0; s < QST; ++s) { mbar_init(&bars.q_full[s], 1); mbar_init(&bars.q_empty[s], 1); }
     for (int s = 0; s < KST; ++s) { mbar_init(&bars.k_full[s], 1); mbar_init(&bars.k_empty[s], 1); }
     for (int s = 0; s < VST; ++s) { mbar_init(&bars.v_full[s], 1); mbar_init(&bars.v_empty[s], 1); }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_free, SOFTMAX_WARPS);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.s_free[s], 4);
-      mbar_init(&bars.p_full[s], 4);
+      mbar_init(&bars.p_full[s][0], SOFTMAX_WARPS / 2);
+      mbar_init(&bars.p_full[s][1], SOFTMAX_WARPS / 2);
       mbar_init(&bars.pv_done[s], 1);
       mbar_init(&bars.item_full[s], 1);
-      mbar_init(&bars.item_empty[s], 5);
+      mbar_init(&bars.item_empty[s], 1 + SOFTMAX_WARPS);
     }
+    mbar_init(&bars.xstate, SOFTMAX_WARPS);
     mbar_init(&bars.o_full, 1);
-    mbar_init(&bars.o_free, 4);
+    mbar_init(&bars.o_free, SOFTMAX_WARPS);
     mbar_init(&bars.teardown, 1);
     bars.abort_flag = 0;
     fence_mbar_init();
@@ -189,159 +217,204 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = bars.tmem_base;
 
   if (warp == 0) {
-    // ================================================================ producer
-    if (lane == 0) {
-      const uint64_t pol_kv = policy_evict_last();
-      const uint64_t pol_q = policy_evict_first();
-      uint32_t g = 0;          // global tile counter
-      int it = 0;              // item counter
-      int k_last_use[KST], v_last_use[VST], q_uses = 0;
-      for (int s = 0; s < KST; ++s) k_last_use[s] = -1;
-      for (int s = 0; s < VST; ++s) v_last_use[s] = -1;
-      bool ok = true;
-      for (;; ++it) {
-        const int slot = it & 1;
-        if (it >= 2 && !(ok = wait_bar(&bars.item_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 1))) break;
-        const int idx = atomicAdd(p.work_counter, 1);
-        const int item = idx < p.nitems ? p.order[idx] : -1;
+    // ================================================================ producer (whole warp, one lane issues)
+    const bool leader = elect_one();
+    const uint64_t pol_kv = policy_evict_last();
+    const uint64_t pol_q = policy_evict_first();
+    uint32_t g = 0;          // global tile counter
+    int k_last_use[KST], v_last_use[VST], q_last_use[QST], q_uses = 0;
+    for (int s = 0; s < KST; ++s) k_last_use[s] = -1;
+    for (int s = 0; s < VST; ++s) v_last_use[s] = -1;
+    for (int s = 0; s < QST; ++s) q_last_use[s] = -1;
+    bool ok = true;
+    for (int it = 0;; ++it) {
+      const int slot = it & 1;
+      if (it >= 2 && !(ok = wait_warp(&bars.item_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 1))) break;
+      int idx = 0;
+      if (lane == 0) idx = atomicAdd(p.work_counter, 1);
+      idx = __shfl_sync(0xffffffffu, idx, 0);
+      const int item = idx < p.nitems ? p.order[idx] : -1;
+      if (lane == 0) {
         bars.item_slot[slot] = item;
         mbar_arrive(&bars.item_full[slot]);
-        if (item < 0) break;
-        const int bh = item / p.N, qi = item % p.N;
-        const int T = p.tiles[item];
-        if (T == 0) continue;
-        if (it > 0 && q_uses > 0 && !(ok = wait_bar(&bars.q_empty, (q_uses - 1) & 1, bars, lim, 2))) break;
-        mbar_arrive_expect_tx(&bars.q_full, TILE_BYTES);
-        tma_load_3d(smem + OFF_Q, &tmQ, &bars.q_full, 0, qi * BM, bh, pol_q);
-        tma_load_3d(smem + OFF_Q + HALF_BYTES, &tmQ, &bars.q_full, 64, qi * BM, bh, pol_q);
-        ++q_uses;
-        TileIter ti;
-        ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.nchunk);
-        int pkind = 0, pidx = 0;
-        for (int n = 0; n <= T && ok; ++n) {
-          int kind = 0, tidx = 0;
-          if (n < T) {
-            ti.next(kind, tidx);
-            const uint32_t gk = g + n;
-            const int ks = gk % KST;
-            if (gk >= KST && !(ok = wait_bar(&bars.k_empty[ks], ((gk / KST) + 1) & 1, bars, lim, 3))) break;
+      }
+      if (item < 0) break;
+      const int bh = item / p.N, qi = item % p.N;
+      const int T = p.tiles[item];
+      if (T == 0) continue;
+      // Q tile into buffer q_uses % QST, once the item that used it last has
+      // issued all its S MMAs
+      const int qb = q_uses % QST;
+      const int qu = q_uses / QST;
+      if (qu > 0 && !(ok = wait_warp(&bars.q_empty[qb], (qu - 1) & 1, bars, lim, 2))) break;
+      if (leader) {
+        mbar_arrive_expect_tx(&bars.q_full[qb], TILE_BYTES);
+        uint8_t* qdst = smem + OFF_Q + qb * TILE_BYTES;
+        tma_load_3d(qdst, &tmQ, &bars.q_full[qb], 0, qi * BM, bh, pol_q);
+        tma_load_3d(qdst + HALF_BYTES, &tmQ, &bars.q_full[qb], 64, qi * BM, bh, pol_q);
+      }
+      q_last_use[qb] = qu;
+      ++q_uses;
+      TileIter ti;
+      ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.nchunk);
+      int pkind = 0, pidx = 0;
+      // K runs one tile ahead of V: K_0, K_1, V_0, K_2, V_1, ...
+      for (int n = 0; n <= T && ok; ++n) {
+        int kind = 0, tidx = 0;
+        if (n < T) {
+          ti.next(kind, tidx);
+          const uint32_t gk = g + n;
+          const int ks = gk % KST;
+          const int ku = gk / KST;
+          if (ku > 0 && !(ok = wait_warp(&bars.k_empty[ks], (ku - 1) & 1, bars, lim, 3))) break;
+          if (leader) {
             uint8_t* dst = smem + OFF_K + ks * TILE_BYTES;
             mbar_arrive_expect_tx(&bars.k_full[ks], TILE_BYTES);
             const CUtensorMap* m = kind ? &tmK : &tmKb;
             tma_load_3d(dst, m, &bars.k_full[ks], 0, tidx * BN, bh, pol_kv);
             tma_load_3d(dst + HALF_BYTES, m, &bars.k_full[ks], 64, tidx * BN, bh, pol_kv);
-            k_last_use[ks] = (int)(gk / KST);
           }
-          if (n > 0) {
-            const uint32_t gv = g + n - 1;
-            const int vs = gv % VST;
-            if (gv >= VST && !(ok = wait_bar(&bars.v_empty[vs], ((gv / VST) + 1) & 1, bars, lim, 4))) break;
+          k_last_use[ks] = ku;
+        }
+        if (n > 0) {
+          const uint32_t gv = g + n - 1;
+          const int vs = gv % VST;
+          const int vu = gv / VST;
+          if (vu > 0 && !(ok = wait_warp(&bars.v_empty[vs], (vu - 1) & 1, bars, lim, 4))) break;
+          if (leader) {
             uint8_t* dst = smem + OFF_V + vs * TILE_BYTES;
             mbar_arrive_expect_tx(&bars.v_full[vs], TILE_BYTES);
             const CUtensorMap* m = pkind ? &tmV : &tmVb;
             tma_load_3d(dst, m, &bars.v_full[vs], 0, pidx * BN, bh, pol_kv);
             tma_load_3d(dst + HALF_BYTES, m, &bars.v_full[vs], 64, pidx * BN, bh, pol_kv);
-            v_last_use[vs] = (int)(gv / VST);
           }
-          pkind = kind;
-          pidx = tidx;
+          v_last_use[vs] = vu;
         }
-        if (!ok) break;
-        g += T;
+        pkind = kind;
+        pidx = tidx;
       }
-      if (!ok || bars.abort_flag) {
-        // let every copy this thread started land before the CTA exits
-        for (int s = 0; s < KST; ++s)
-          if (k_last_use[s] >= 0) mbar_wait(&bars.k_full[s], k_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
-        for (int s = 0; s < VST; ++s)
-          if (v_last_use[s] >= 0) mbar_wait(&bars.v_full[s], v_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
-        if (q_uses > 0) mbar_wait(&bars.q_full, (q_uses - 1) & 1, nullptr, &g_sol_status, 0, lim);
-      }
+      if (!ok) break;
+      g += T;
+    }
+    if (!ok || bars.abort_flag) {
+      // let every copy this warp started land before the CTA exits
+      for (int s = 0; s < KST; ++s)
+        if (k_last_use[s] >= 0) mbar_wait(&bars.k_full[s], k_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
+      for (int s = 0; s < VST; ++s)
+        if (v_last_use[s] >= 0) mbar_wait(&bars.v_full[s], v_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
+      for (int s = 0; s < QST; ++s)
+        if (q_last_use[s] >= 0) mbar_wait(&bars.q_full[s], q_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-      const uint32_t sQ = smem_u32(smem + OFF_Q);
-      const uint32_t sK = smem_u32(smem + OFF_K);
-      const uint32_t sV = smem_u32(smem + OFF_V);
-      uint32_t g = 0;
-      int item_local = 0;  // items with T > 0 processed
-      bool issued = false;
-      bool ok = true;
-      for (int it = 0;; ++it) {
-        const int slot = it & 1;
-        if (!(ok = wait_bar(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 10))) break;
-        const int item = bars.item_slot[slot];
-        mbar_arrive(&bars.item_empty[slot]);
-        if (item < 0) break;
-        const int T = p.tiles[item];
-        if (T == 0) continue;
-        if (!(ok = wait_bar(&bars.q_full, item_local & 1, bars, lim, 11))) break;
-        auto issue_pv = [&](uint32_t gp, bool first) -> bool {
-          const int pb = gp & 1;
-          if (!wait_bar(&bars.p_full[pb], (gp >> 1) & 1, bars, lim, 12)) return false;
-          const int vs = gp % VST;
-          if (!wait_bar(&bars.v_full[vs], (gp / VST) & 1, bars, lim, 13)) return false;
-          if (first && item_local > 0 && !wait_bar(&bars.o_free, (item_local - 1) & 1, bars, lim, 14)) return false;
-          tc_fence_after();
-          const uint32_t vbase = sV + vs * TILE_BYTES;
+    // ================================================================ MMA issuer (whole warp, one lane issues)
+    const bool leader = elect_one();
+    constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+    constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
+    const uint32_t sK = smem_u32(smem + OFF_K);
+    const uint32_t sV = smem_u32(smem + OFF_V);
+    uint32_t g = 0;
+    int item_local = 0;  // items with T > 0 processed
+    bool issued = false;
+    bool ok = true;
+    // S_gs = Q K_gs^T into the single S buffer, once the softmax has read S_{gs-1}
+    auto issue_s = [&](uint32_t gs, uint32_t sQ) -> bool {
+      const int ks = gs % KST;
+      if (!wait_warp(&bars.k_full[ks], (gs / KST) & 1, bars, lim, 15)) return false;
+      if (gs >= 1 && !wait_warp(&bars.s_free, (gs - 1) & 1, bars, lim, 16)) return false;
+      tc_fence_after();
+      const uint32_t kbase = sK + ks * TILE_BYTES;
+      if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, HALF_BYTES, 1024);
-            mma_ts(tmem + TM_O, tmem + TM_P + pb * 64 + kk * 8, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
-          }
-          tc_commit(&bars.v_empty[vs]);
-          tc_commit(&bars.pv_done[pb]);
-          return true;
-        };
-        for (int n = 0; n < T && ok; ++n) {
-          const uint32_t gs = g + n;
-          const int ks = gs % KST;
-          if (!(ok = wait_bar(&bars.k_full[ks], (gs / KST) & 1, bars, lim, 15))) break;
-          const int sb = gs & 1;
-          if (gs >= 2 && !(ok = wait_bar(&bars.s_free[sb], ((gs >> 1) + 1) & 1, bars, lim, 16))) break;
-          tc_fence_after();
-          const uint32_t kbase = sK + ks * TILE_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            const uint64_t adesc = smem_desc_sw128(sQ + off, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(kbase + off, 16, 1024);
-            mma_ss(tmem + TM_S + sb * 128, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          issued = true;
-          tc_commit(&bars.s_full[sb]);
-          tc_commit(&bars.k_empty[ks]);
-          if (n == T - 1) tc_commit(&bars.q_empty);
-          if (n > 0 && !(ok = issue_pv(gs - 1, n == 1))) break;
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + TM_S, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                 IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        if (!ok) break;
-        if (!(ok = issue_pv(g + T - 1, T == 1))) break;
-        tc_commit(&bars.o_full);
-        g += T;
-        ++item_local;
+        tc_commit(&bars.s_full);
+        tc_commit(&bars.k_empty[ks]);
       }
-      if (issued) {
-        // all MMAs of this CTA complete before TMEM is released
-        tc_commit(&bars.teardown);
-        mbar_wait(&bars.teardown, 0, nullptr, &g_sol_status, 0, lim);
+      __syncwarp();
+      return true;
+    };
+    // O_h += P_h V_h for both halves of tile gp
+    auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+      const int pb = gp & 1;
+      const int vs = gp % VST;
+      if (!wait_warp(&bars.v_full[vs], (gp / VST) & 1, bars, lim, 13)) return false;
+      if (first && item_local > 0 && !wait_warp(&bars.o_free, (item_local - 1) & 1, bars, lim, 14)) return false;
+      const uint32_t vbase = sV + vs * TILE_BYTES;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (!wait_warp(&bars.p_full[pb][h], (gp >> 1) & 1, bars, lim, 12)) return false;
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tmem + TM_O + h * 128, tmem + TM_P + pb * 64 + h * 32 + kk * 8,
+                   smem_desc_sw128(vbase + h * 8192 + kk * 2048, HALF_BYTES, 1024), IDESC_PV,
+                   (first && kk == 0) ? 0u : 1u);
+        }
+        __syncwarp();
       }
+      if (leader) {
+        tc_commit(&bars.v_empty[vs]);
+        tc_commit(&bars.pv_done[pb]);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int it = 0;; ++it) {
+      const int slot = it & 1;
+      if (!(ok = wait_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 10))) break;
+      const int item = bars.item_slot[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
+      if (item < 0) break;
+      const int T = p.tiles[item];
+      if (T == 0) continue;
+      const int qb = item_local % QST;
+      if (!(ok = wait_warp(&bars.q_full[qb], (item_local / QST) & 1, bars, lim, 11))) break;
+      const uint32_t sQ = smem_u32(smem + OFF_Q + qb * TILE_BYTES);
+      // order: S_0, then for each tile n: S_{n+1}, PV_n
+      if (!(ok = issue_s(g, sQ))) break;
+      issued = true;
+      for (int n = 0; n < T && ok; ++n) {
+        if (n + 1 < T) {
+          if (!(ok = issue_s(g + n + 1, sQ))) break;
+        } else if (leader) {
+          tc_commit(&bars.q_empty[qb]);  // every S MMA of this item has been issued
+        }
+        if (!(ok = issue_pv(g + n, n == 0))) break;
+      }
+      if (!ok) break;
+      if (leader) tc_commit(&bars.o_full);
+      __syncwarp();
+      g += T;
+      ++item_local;
+    }
+    if (issued) {
+      // all MMAs of this CTA complete before TMEM is released
+      if (leader) tc_commit(&bars.teardown);
+      __syncwarp();
+      mbar_wait(&bars.teardown, 0, nullptr, &g_sol_status, 0, lim);
     }
     __syncwarp();
   } else {
     // ================================================================ softmax + epilogue
-    const int quad = warp & 3;           // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;    // query row within the tile
+    const int half = (warp - 2) >> 2;     // column half of every S tile this warp owns
+    const int quad = warp & 3;            // TMEM lane quadrant this warp may access
+    const int row = quad * 32 + lane;     // query row within the tile
+    const int col0 = half * 64;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tO = tmem + lane_off + TM_O + half * 128;  // this half's accumulator O_h
+    const float sl2 = p.scale_log2;
     uint32_t g = 0;
     int item_local = 0;
     bool ok = true;
     for (int it = 0;; ++it) {
       const int slot = it & 1;
-      if (!(ok = wait_bar_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 20))) break;
+      if (!(ok = wait_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 20))) break;
       const int item = bars.item_slot[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
@@ -349,10 +422,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int bh = item / p.N, qi = item % p.N;
       const int T = p.tiles[item];
       const int n_rows = min(BM, p.L - qi * BM);
-      __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD;
+      __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD + col0;
       if (T == 0) {
         if (row < n_rows)
-          for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 64; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
       TileIter ti;
@@ -362,56 +435,66 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int kind = 0, tidx = 0;
         ti.next(kind, tidx);
         const uint32_t gs = g + n;
-        const int sb = gs & 1;
-        if (!(ok = wait_bar_warp(&bars.s_full[sb], (gs >> 1) & 1, bars, lim, 21))) break;
+        const int pb = gs & 1;
+        if (!(ok = wait_warp(&bars.s_full, gs & 1, bars, lim, 21))) break;
         tc_fence_after();
-        float x[128];
+        float x[64];
         {
-          uint32_t r[32];
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tmem + lane_off + TM_S + col0, r0);
+          tmem_ld32(tmem + lane_off + TM_S + col0 + 32, r1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            tmem_ld32(tmem + lane_off + TM_S + sb * 128 + q * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) x[q * 32 + c] = __uint_as_float(r[c]);
+          for (int c = 0; c < 32; ++c) {
+            x[c] = __uint_as_float(r0[c]);
+            x[32 + c] = __uint_as_float(r1[c]);
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.s_free[sb]);
+        if (lane == 0) mbar_arrive(&bars.s_free);
 
-        // column validity and bias of this tile
-        float rmax;
-        if (kind == 1 && (tidx != p.N - 1 || p.n_last == BN)) {
-          const uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
-          rmax = tile_logits<true>(x, p.scale_log2, 0.f, vm, -1, 0.f);
+        // full exact tile: x stays the raw score (scale folded into exp2 below);
+        // otherwise x becomes the log2-domain logit with bias and mask applied
+        const bool full = kind == 1 && (tidx != p.N - 1 || p.n_last == BN);
+        float lmax;
+        if (full) {
+          lmax = tree_max64(x) * sl2;  // scaling by sl2 > 0 commutes with max
         } else {
-          uint32_t vm[4];
+          uint32_t vm[2];
           float bias = 0.f;
           int sc = -1;
           float sc_delta = 0.f;
           if (kind == 1) {  // partial last key block: columns >= n_last are padding
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int nb = p.n_last - q * 32;
+            for (int q = 0; q < 2; ++q) {
+              const int nb = p.n_last - col0 - q * 32;
               vm[q] = nb >= 32 ? ~0u : (nb <= 0 ? 0u : ((1u << nb) - 1u));
             }
           } else {  // pooled chunk: unselected, in-range blocks only
             bias = p.bias_full;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int w = tidx * 4 + q;
+            for (int q = 0; q < 2; ++q) {
+              const int w = tidx * 4 + half * 2 + q;
               vm[q] = (w < p.W) ? ((~p.mask[(size_t)item * p.W + w]) & ti.valid_bits(w)) : 0u;
             }
-            const int jl = p.N - 1 - tidx * BN;
-            if (jl >= 0 && jl < BN && p.n_last != BN) {
+            const int jl = p.N - 1 - tidx * BN - col0;
+            if (jl >= 0 && jl < 64 && p.n_last != BN) {
               sc = jl;
               sc_delta = p.bias_last - p.bias_full;
             }
           }
-          rmax = tile_logits<false>(x, p.scale_log2, bias, vm, sc, sc_delta);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            float u = fmaf(x[c], sl2, bias);
+            if (c == sc) u += sc_delta;
+            x[c] = ((vm[c >> 5] >> (c & 31)) & 1u) ? u : -INFINITY;
+          }
+          lmax = tree_max64(x);
         }
-        const float m_new = fmaxf(m_used, rmax);
+        // this half's running max (a half may see only masked columns: it
+        // then keeps m = -inf and all its probabilities are 0)
+        const float m_new = fmaxf(m_used, lmax);
         const bool need = m_new > m_used + RESCALE_THRESHOLD;
         float alpha = 1.f;
         if (need) {
@@ -419,62 +502,93 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           m_used = m_new;
           l *= alpha;
         }
-        uint32_t pk[2][32];
-        float rs = 0.f;
+        const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+        const float2 sl2v = make_float2(full ? sl2 : 1.f, full ? sl2 : 1.f);
+        const float2 negv = make_float2(neg_m, neg_m);
+        uint32_t pk[32];
+        float2 acc[4];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = ex2_approx(x[c] - m_used);
-          const float p1 = ex2_approx(x[c + 1] - m_used);
-          rs += p0 + p1;
-          pk[c >> 6][(c & 63) >> 1] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float2 a = fma2(make_float2(x[c], x[c + 1]), sl2v, negv);
+          float2 e;
+          if (((c >> 1) % POLY_PAIR_PERIOD) == POLY_PAIR_PERIOD - 1) {
+            e = exp2_poly2(a);
+          } else {
+            e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+          }
+          acc[(c >> 1) & 3] = add2(acc[(c >> 1) & 3], e);
+          pk[c >> 1] = pack_bf16x2(e.x, e.y);
         }
-        l += rs;
-        // P buffer sb was read by the PV of tile gs - 2
-        if (gs >= 2 && !(ok = wait_bar_warp(&bars.pv_done[sb], ((gs - 2) >> 1) & 1, bars, lim, 22))) break;
-        tmem_st32(tmem + lane_off + TM_P + sb * 64, pk[0]);
-        tmem_st32(tmem + lane_off + TM_P + sb * 64 + 32, pk[1]);
+        const float2 s2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+        l += s2.x + s2.y;
+        // P buffer pb was read by the PV of tile gs - 2
+        if (gs >= 2 && !(ok = wait_warp(&bars.pv_done[pb], ((gs - 2) >> 1) & 1, bars, lim, 22))) break;
+        tmem_st32(tmem + lane_off + TM_P + pb * 64 + half * 32, pk);
         if (n > 0 && __any_sync(0xffffffffu, need)) {
-          // O must hold every PV up to tile gs - 1 before it is rescaled
+          // O_h must hold every PV up to tile gs - 1 before it is rescaled
           const uint32_t gp = gs - 1;
-          if (!(ok = wait_bar_warp(&bars.pv_done[gp & 1], (gp >> 1) & 1, bars, lim, 23))) break;
+          if (!(ok = wait_warp(&bars.pv_done[gp & 1], (gp >> 1) & 1, bars, lim, 23))) break;
           tc_fence_after();
-          uint32_t o[32];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            tmem_ld32(tmem + lane_off + TM_O + q * 32, o);
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tmem + lane_off + TM_O + q * 32, o);
+            tmem_st32(tO + q * 32, o);
           }
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[sb]);
+        if (lane == 0) mbar_arrive(&bars.p_full[pb][half]);
       }
       if (!ok) break;
-      // epilogue: O / l for this row
-      if (!(ok = wait_bar_warp(&bars.o_full, item_local & 1, bars, lim, 24))) break;
+      // epilogue: merge the two halves' softmax states, write this half's 64
+      // output columns: out = (O_0 e_0 + O_1 e_1) / (l_0 e_0 + l_1 e_1),
+      // e_h = 2^(m_h - max(m_0, m_1))
+      // (double-buffered by item: a half may finish the next item's key loop
+      // before its partner has read this item's state)
+      const int xb = item_local & 1;
+      bars.xm[xb][half][row] = m_used;
+      bars.xl[xb][half][row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.xstate);
+      if (!(ok = wait_warp(&bars.o_full, item_local & 1, bars, lim, 24))) break;
       tc_fence_after();
-      const float inv = 1.0f / l;
-      uint32_t ob[4][32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tmem + lane_off + TM_O + q * 32, ob[q]);
+      uint32_t o0[2][32], o1[2][32];
+      tmem_ld32(tmem + lane_off + TM_O + col0, o0[0]);
+      tmem_ld32(tmem + lane_off + TM_O + col0 + 32, o0[1]);
+      tmem_ld32(tmem + lane_off + TM_O + 128 + col0, o1[0]);
+      tmem_ld32(tmem + lane_off + TM_O + 128 + col0 + 32, o1[1]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.o_free);
+      if (!(ok = wait_warp(&bars.xstate, item_local & 1, bars, lim, 26))) break;
+      const float m0 = bars.xm[xb][0][row], m1 = bars.xm[xb][1][row];
+      const float mm = fmaxf(m0, m1);
+      const float e0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
+      const float e1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
+      const float inv = 1.0f / (bars.xl[xb][0][row] * e0 + bars.xl[xb][1][row] * e1);
+      const float w0 = e0 * inv, w1 = e1 * inv;
       if (row < n_rows) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              v[e] = __uint_as_float(o0[q][c + e]) * w0 + __uint_as_float(o1[q][c + e]) * w1;
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ob[q][c + 0]) * inv, __uint_as_float(ob[q][c + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ob[q][c + 2]) * inv, __uint_as_float(ob[q][c + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ob[q][c + 4]) * inv, __uint_as_float(ob[q][c + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ob[q][c + 6]) * inv, __uint_as_float(ob[q][c + 7]) * inv);
+            w.x = pack_bf16x2(v[0], v[1]);
+            w.y = pack_bf16x2(v[2], v[3]);
+            w.z = pack_bf16x2(v[4], v[5]);
+            w.w = pack_bf16x2(v[6], v[7]);
             *reinterpret_cast<uint4*>(orow + q * 32 + c) = w;
           }
         }
