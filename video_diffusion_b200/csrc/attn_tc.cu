@@ -92,6 +92,7 @@ struct Bars {
   float xl[2][2][BM];     // [item parity][column half][row] row sum
 };
 static_assert(sizeof(Bars) <= BAR_AREA, "barrier area");
+static_assert(KST == 2 && VST == 2 && QST == 2, "the producer's abort path assumes 2-deep rings");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
 // unselected block, then the selected blocks in increasing order.
@@ -222,10 +223,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
     uint32_t g = 0;          // global tile counter
-    int k_last_use[KST], v_last_use[VST], q_last_use[QST], q_uses = 0;
-    for (int s = 0; s < KST; ++s) k_last_use[s] = -1;
-    for (int s = 0; s < VST; ++s) v_last_use[s] = -1;
-    for (int s = 0; s < QST; ++s) q_last_use[s] = -1;
+    // last K / V tile and number of Q tiles whose loads were issued (to let
+    // them land if the CTA abandons its work)
+    int gk_last = -1, gv_last = -1, q_uses = 0;
     bool ok = true;
     for (int it = 0;; ++it) {
       const int slot = it & 1;
@@ -253,7 +253,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_load_3d(qdst, &tmQ, &bars.q_full[qb], 0, qi * BM, bh, pol_q);
         tma_load_3d(qdst + HALF_BYTES, &tmQ, &bars.q_full[qb], 64, qi * BM, bh, pol_q);
       }
-      q_last_use[qb] = qu;
       ++q_uses;
       TileIter ti;
       ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.nchunk);
@@ -274,7 +273,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_3d(dst, m, &bars.k_full[ks], 0, tidx * BN, bh, pol_kv);
             tma_load_3d(dst + HALF_BYTES, m, &bars.k_full[ks], 64, tidx * BN, bh, pol_kv);
           }
-          k_last_use[ks] = ku;
+          gk_last = (int)gk;
         }
         if (n > 0) {
           const uint32_t gv = g + n - 1;
@@ -288,7 +287,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_3d(dst, m, &bars.v_full[vs], 0, pidx * BN, bh, pol_kv);
             tma_load_3d(dst + HALF_BYTES, m, &bars.v_full[vs], 64, pidx * BN, bh, pol_kv);
           }
-          v_last_use[vs] = vu;
+          gv_last = (int)gv;
         }
         pkind = kind;
         pidx = tidx;
@@ -297,13 +296,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       g += T;
     }
     if (!ok || bars.abort_flag) {
-      // let every copy this warp started land before the CTA exits
-      for (int s = 0; s < KST; ++s)
-        if (k_last_use[s] >= 0) mbar_wait(&bars.k_full[s], k_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
-      for (int s = 0; s < VST; ++s)
-        if (v_last_use[s] >= 0) mbar_wait(&bars.v_full[s], v_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
-      for (int s = 0; s < QST; ++s)
-        if (q_last_use[s] >= 0) mbar_wait(&bars.q_full[s], q_last_use[s] & 1, nullptr, &g_sol_status, 0, lim);
+      // let every copy this warp started land before the CTA exits: the last
+      // use of each 2-deep ring stage is one of the last two issued tiles
+      for (int back = 0; back < 2; ++back) {
+        const int gk = gk_last - back, gv = gv_last - back, qu = q_uses - 1 - back;
+        if (gk >= 0) mbar_wait(&bars.k_full[gk % KST], (gk / KST) & 1, nullptr, &g_sol_status, 0, lim);
+        if (gv >= 0) mbar_wait(&bars.v_full[gv % VST], (gv / VST) & 1, nullptr, &g_sol_status, 0, lim);
+        if (qu >= 0) mbar_wait(&bars.q_full[qu % QST], (qu / QST) & 1, nullptr, &g_sol_status, 0, lim);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {

@@ -104,17 +104,19 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict_
 constexpr int kRouteThreads = 256;
 constexpr int kRouteKC = 32;  // pooled keys staged in shared memory at a time
 
-// grid (ceil(N / QB), bH), 256 threads.  Each warp owns one query block of
-// the group for the row statistics; the score pass pairs warp w with query
-// block w and lane l with key l of the staged chunk.
-template <int D>
+// grid (ceil(N / QB), bH), 256 threads, QB a multiple of 8 (up to 32).
+// Score pass: lane l takes staged key l, warp w the query blocks
+// w*QB/8 .. (w+1)*QB/8 - 1, so each thread runs QB/8 independent dot
+// products over one key row.  Row pass: warp w takes query blocks w, w + 8, ...
+template <int D, int QPW>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __restrict__ qbar,
                                                               const float* __restrict__ kbar, int N, int W,
-                                                              int B, int nchunk, int QB, float scale, float beta,
+                                                              int B, int nchunk, float scale, float beta,
                                                               int beta_mode, int correction,
                                                               uint32_t* __restrict__ mask,
                                                               int32_t* __restrict__ counts,
                                                               int32_t* __restrict__ tiles) {
+  constexpr int QB = 8 * QPW;
   extern __shared__ float sm[];
   float* qs = sm;                          // [QB][D]
   float* ks = qs + QB * D;                 // [KC][D + 1]
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
   const float* qb = qbar + ((size_t)bh * N + i0) * D;
   const float* kb = kbar + (size_t)bh * N * D;
 
-  for (int e = tid; e < nq * D; e += kRouteThreads) qs[e] = qb[e];
+  for (int e = tid; e < QB * D; e += kRouteThreads) qs[e] = e < nq * D ? qb[e] : 0.f;
   for (int j0 = 0; j0 < N; j0 += kRouteKC) {
     const int nk = min(kRouteKC, N - j0);
     __syncthreads();
@@ -135,14 +137,22 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
       ks[jj * (D + 1) + c] = kb[(size_t)(j0 + jj) * D + c];
     }
     __syncthreads();
-    for (int qi = warp; qi < nq; qi += kRouteThreads / 32) {
-      if (lane < nk) {
-        const float* qv = qs + qi * D;
-        const float* kv = ks + lane * (D + 1);
-        float s = 0.f;
-#pragma unroll 16
-        for (int c = 0; c < D; ++c) s = fmaf(qv[c], kv[c], s);
-        srow[(size_t)qi * N + j0 + lane] = s * scale;
+    if (lane < nk) {
+      const float* kv = ks + lane * (D + 1);
+      const float* qv = qs + warp * QPW * D;
+      float acc[QPW];
+#pragma unroll
+      for (int q = 0; q < QPW; ++q) acc[q] = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) {
+        const float kc = kv[c];
+#pragma unroll
+        for (int q = 0; q < QPW; ++q) acc[q] = fmaf(qv[q * D + c], kc, acc[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < QPW; ++q) {
+        const int qi = warp * QPW + q;
+        if (qi < nq) srow[(size_t)qi * N + j0 + lane] = acc[q] * scale;
       }
     }
   }
@@ -276,32 +286,39 @@ cudaError_t launch_pool(int in_dtype, int op_dtype, const void* q, const void* k
   return pool_dispatch<float, __nv_bfloat16>(q, k, v, g, s, st);
 }
 
-static int route_qb(int N) {
-  // query blocks per CTA, bounded by the shared memory their score rows take
-  int qb = 8;
-  while (qb > 1 && (size_t)qb * N * sizeof(float) > 160u * 1024u) qb >>= 1;
-  return qb;
+// Query blocks per CTA (QB = 8 * QPW), bounded by the shared memory their
+// score rows take.
+static int route_qpw(int N) {
+  int qpw = 4;
+  while (qpw > 1 && (size_t)8 * qpw * N * sizeof(float) > 160u * 1024u) qpw >>= 1;
+  return qpw;
+}
+
+template <int D, int QPW>
+static cudaError_t route_launch(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
+                                cudaStream_t st) {
+  constexpr int QB = 8 * QPW;
+  const size_t smem = (size_t)(QB * D + kRouteKC * (D + 1) + (size_t)QB * g.N) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, QPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((g.N + QB - 1) / QB, g.bH);
+  route_kernel<D, QPW><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, g.N, g.W, g.B, g.nchunk,
+                                                          1.0f / sqrtf((float)D), beta, beta_mode, correction,
+                                                          s.mask, s.counts, s.tiles);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_route(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
                          cudaStream_t st) {
-  const int QB = route_qb(g.N);
-  const size_t smem = (size_t)(QB * g.d + kRouteKC * (g.d + 1) + (size_t)QB * g.N) * sizeof(float);
-  dim3 grid((g.N + QB - 1) / QB, g.bH);
-  const float scale = 1.0f / sqrtf((float)g.d);
-  cudaError_t e;
+  const int qpw = route_qpw(g.N);
   if (g.d == 128) {
-    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<128><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, g.N, g.W, g.B, g.nchunk, QB, scale, beta,
-                                                         beta_mode, correction, s.mask, s.counts, s.tiles);
-  } else {
-    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<64><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, g.N, g.W, g.B, g.nchunk, QB, scale, beta,
-                                                        beta_mode, correction, s.mask, s.counts, s.tiles);
+    if (qpw == 4) return route_launch<128, 4>(g, s, beta, beta_mode, correction, st);
+    if (qpw == 2) return route_launch<128, 2>(g, s, beta, beta_mode, correction, st);
+    return route_launch<128, 1>(g, s, beta, beta_mode, correction, st);
   }
-  return cudaGetLastError();
+  if (qpw == 4) return route_launch<64, 4>(g, s, beta, beta_mode, correction, st);
+  if (qpw == 2) return route_launch<64, 2>(g, s, beta, beta_mode, correction, st);
+  return route_launch<64, 1>(g, s, beta, beta_mode, correction, st);
 }
 
 cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st) {
