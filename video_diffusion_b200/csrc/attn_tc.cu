@@ -1,6 +1,11 @@
 // attn_tc.cu -- the Sol-Attn attention loop on the 5th-generation tensor cores
 // (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, d = 128, B = 128.
 //
+// The MMA warp's barrier operations, not the tensor pipe, set the pace of
+// the key loop (each wait or commit costs a few hundred cycles while the
+// softmax warps keep the memory pipes busy), so the handoffs per tile are
+// kept to three waits and three commits.
+//
 // One online-softmax pass per query block i (Sol-Attn visual explainer, "One
 // online-softmax state": exact and approximate terms share the running
 // maximum, the denominator and the numerator):
@@ -14,8 +19,10 @@
 //     Only selected K/V tiles are ever loaded.
 //
 // Persistent CTAs, one per SM, 320 threads:
-//   warp 0      TMA producer: fetches work items, loads Q tiles (2 buffers)
-//               and K/V (or K-bar/V-bar) tiles (2-stage K and V rings)
+//   warp 0      TMA producer: fetches work items, loads the Q tile and each
+//               tile's K and V (or K-bar and V-bar) together into a 3-stage
+//               ring (a tile copy takes about a tile's worth of time when
+//               every SM loads at once, so copies run up to three tiles ahead)
 //   warp 1      TMEM owner and tcgen05.mma issuer (one elected lane)
 //   warps 2..9  softmax, two column halves: half h owns the 64 keys
 //               [64h, 64h + 64) of every tile, one query row per thread (its
@@ -41,17 +48,19 @@ __device__ int g_sol_status;  // 0 = ok; else 0x1000 | wait id (first expiry)
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int QST = 2, KST = 2, VST = 2;
+constexpr int QST = 1, KVST = 3;  // Q buffers, K+V stages
 constexpr int NTHREADS = 320;
 constexpr int SOFTMAX_WARPS = 8;
 constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB, two 64-column swizzled halves
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + QST * TILE_BYTES;
-constexpr uint32_t OFF_V = OFF_K + KST * TILE_BYTES;
-constexpr uint32_t OFF_BAR = OFF_V + VST * TILE_BYTES;  // 192 KB
-constexpr uint32_t BAR_AREA = 8192;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA + 1024;  // + alignment slack
+constexpr uint32_t OFF_KV = OFF_Q + QST * TILE_BYTES;  // stage s: K at +2s tiles, V at +2s+1
+constexpr uint32_t OFF_BAR = OFF_KV + 2 * KVST * TILE_BYTES;  // 224 KB
+constexpr uint32_t BAR_AREA = 2560;
+// No room for alignment slack: the kernel checks that dynamic shared memory
+// starts on a 1024-byte boundary (the 128-byte swizzle needs it) and reports
+// an error instead of running if it does not.
+constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA;
 
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_P = 384;  // O_h at TM_O + 128 h
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -76,23 +85,23 @@ struct Params {
 
 struct Bars {
   uint64_t q_full[QST], q_empty[QST];
-  uint64_t k_full[KST], k_empty[KST];
-  uint64_t v_full[VST], v_empty[VST];
+  uint64_t kv_full[KVST], kv_empty[KVST];
   uint64_t s_full, s_free;
-  uint64_t p_full[2][2];  // [P buffer][column half]
+  uint64_t p_full[2];     // [P buffer]: both column halves have written P
   uint64_t pv_done[2];    // per P buffer: both PV MMAs that read it have finished
   uint64_t o_full, o_free;
   uint64_t item_full[2], item_empty[2];
   uint64_t xstate;        // softmax-state exchange between the halves at the end of an item
+  uint64_t xread;         // both halves have read the exchanged state
   uint64_t teardown;
   int item_slot[2];
   uint32_t tmem_base;
   int abort_flag;
-  float xm[2][2][BM];     // [item parity][column half][row] running max (log2 units)
-  float xl[2][2][BM];     // [item parity][column half][row] row sum
+  float xm[2][BM];        // [column half][row] running max (log2 units)
+  float xl[2][BM];        // [column half][row] row sum
 };
 static_assert(sizeof(Bars) <= BAR_AREA, "barrier area");
-static_assert(KST == 2 && VST == 2 && QST == 2, "the producer's abort path assumes 2-deep rings");
+static_assert(QST == 1, "one Q buffer");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
 // unselected block, then the selected blocks in increasing order.
@@ -178,26 +187,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                    const __grid_constant__ CUtensorMap tmVb, const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(&g_sol_status, 0, 0x2000);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   Bars& bars = *reinterpret_cast<Bars*>(smem + OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < QST; ++s) { mbar_init(&bars.q_full[s], 1); mbar_init(&bars.q_empty[s], 1); }
-    for (int s = 0; s < KST; ++s) { mbar_init(&bars.k_full[s], 1); mbar_init(&bars.k_empty[s], 1); }
-    for (int s = 0; s < VST; ++s) { mbar_init(&bars.v_full[s], 1); mbar_init(&bars.v_empty[s], 1); }
+    for (int s = 0; s < KVST; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
     mbar_init(&bars.s_full, 1);
     mbar_init(&bars.s_free, SOFTMAX_WARPS);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.p_full[s][0], SOFTMAX_WARPS / 2);
-      mbar_init(&bars.p_full[s][1], SOFTMAX_WARPS / 2);
+      mbar_init(&bars.p_full[s], SOFTMAX_WARPS);
       mbar_init(&bars.pv_done[s], 1);
       mbar_init(&bars.item_full[s], 1);
       mbar_init(&bars.item_empty[s], 1 + SOFTMAX_WARPS);
     }
     mbar_init(&bars.xstate, SOFTMAX_WARPS);
+    mbar_init(&bars.xread, SOFTMAX_WARPS);
     mbar_init(&bars.o_full, 1);
     mbar_init(&bars.o_free, SOFTMAX_WARPS);
     mbar_init(&bars.teardown, 1);
@@ -225,7 +237,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t g = 0;          // global tile counter
     // last K / V tile and number of Q tiles whose loads were issued (to let
     // them land if the CTA abandons its work)
-    int gk_last = -1, gv_last = -1, q_uses = 0;
+    int gk_last = -1, q_uses = 0;
     bool ok = true;
     for (int it = 0;; ++it) {
       const int slot = it & 1;
@@ -256,54 +268,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ++q_uses;
       TileIter ti;
       ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.nchunk);
-      int pkind = 0, pidx = 0;
-      // K runs one tile ahead of V: K_0, K_1, V_0, K_2, V_1, ...
-      for (int n = 0; n <= T && ok; ++n) {
+      for (int n = 0; n < T; ++n) {
         int kind = 0, tidx = 0;
-        if (n < T) {
-          ti.next(kind, tidx);
-          const uint32_t gk = g + n;
-          const int ks = gk % KST;
-          const int ku = gk / KST;
-          if (ku > 0 && !(ok = wait_warp(&bars.k_empty[ks], (ku - 1) & 1, bars, lim, 3))) break;
-          if (leader) {
-            uint8_t* dst = smem + OFF_K + ks * TILE_BYTES;
-            mbar_arrive_expect_tx(&bars.k_full[ks], TILE_BYTES);
-            const CUtensorMap* m = kind ? &tmK : &tmKb;
-            tma_load_3d(dst, m, &bars.k_full[ks], 0, tidx * BN, bh, pol_kv);
-            tma_load_3d(dst + HALF_BYTES, m, &bars.k_full[ks], 64, tidx * BN, bh, pol_kv);
-          }
-          gk_last = (int)gk;
+        ti.next(kind, tidx);
+        const uint32_t gk = g + n;
+        const int ks = gk % KVST;
+        const int ku = gk / KVST;
+        // stage ks is free once the PV of its previous tile has finished
+        if (ku > 0 && !(ok = wait_warp(&bars.kv_empty[ks], (ku - 1) & 1, bars, lim, 3))) break;
+        if (leader) {
+          uint8_t* dk = smem + OFF_KV + (2 * ks) * TILE_BYTES;
+          uint8_t* dv = dk + TILE_BYTES;
+          mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
+          const CUtensorMap* mk = kind ? &tmK : &tmKb;
+          const CUtensorMap* mv = kind ? &tmV : &tmVb;
+          tma_load_3d(dk, mk, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
+          tma_load_3d(dk + HALF_BYTES, mk, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
+          tma_load_3d(dv, mv, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
+          tma_load_3d(dv + HALF_BYTES, mv, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
         }
-        if (n > 0) {
-          const uint32_t gv = g + n - 1;
-          const int vs = gv % VST;
-          const int vu = gv / VST;
-          if (vu > 0 && !(ok = wait_warp(&bars.v_empty[vs], (vu - 1) & 1, bars, lim, 4))) break;
-          if (leader) {
-            uint8_t* dst = smem + OFF_V + vs * TILE_BYTES;
-            mbar_arrive_expect_tx(&bars.v_full[vs], TILE_BYTES);
-            const CUtensorMap* m = pkind ? &tmV : &tmVb;
-            tma_load_3d(dst, m, &bars.v_full[vs], 0, pidx * BN, bh, pol_kv);
-            tma_load_3d(dst + HALF_BYTES, m, &bars.v_full[vs], 64, pidx * BN, bh, pol_kv);
-          }
-          gv_last = (int)gv;
-        }
-        pkind = kind;
-        pidx = tidx;
+        gk_last = (int)gk;
       }
       if (!ok) break;
       g += T;
     }
     if (!ok || bars.abort_flag) {
       // let every copy this warp started land before the CTA exits: the last
-      // use of each 2-deep ring stage is one of the last two issued tiles
-      for (int back = 0; back < 2; ++back) {
-        const int gk = gk_last - back, gv = gv_last - back, qu = q_uses - 1 - back;
-        if (gk >= 0) mbar_wait(&bars.k_full[gk % KST], (gk / KST) & 1, nullptr, &g_sol_status, 0, lim);
-        if (gv >= 0) mbar_wait(&bars.v_full[gv % VST], (gv / VST) & 1, nullptr, &g_sol_status, 0, lim);
-        if (qu >= 0) mbar_wait(&bars.q_full[qu % QST], (qu / QST) & 1, nullptr, &g_sol_status, 0, lim);
+      // use of each ring stage is one of the ring's last issued tiles
+      for (int back = 0; back < KVST; ++back) {
+        const int gk = gk_last - back;
+        if (gk >= 0) mbar_wait(&bars.kv_full[gk % KVST], (gk / KVST) & 1, nullptr, &g_sol_status, 0, lim);
       }
+      if (q_uses > 0) mbar_wait(&bars.q_full[0], (q_uses - 1) & 1, nullptr, &g_sol_status, 0, lim);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -311,19 +307,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const bool leader = elect_one();
     constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-    const uint32_t sK = smem_u32(smem + OFF_K);
-    const uint32_t sV = smem_u32(smem + OFF_V);
+    const uint32_t sKV = smem_u32(smem + OFF_KV);
     uint32_t g = 0;
     int item_local = 0;  // items with T > 0 processed
     bool issued = false;
     bool ok = true;
     // S_gs = Q K_gs^T into the single S buffer, once the softmax has read S_{gs-1}
     auto issue_s = [&](uint32_t gs, uint32_t sQ) -> bool {
-      const int ks = gs % KST;
-      if (!wait_warp(&bars.k_full[ks], (gs / KST) & 1, bars, lim, 15)) return false;
+      const int ks = gs % KVST;
+      if (!wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 15)) return false;
       if (gs >= 1 && !wait_warp(&bars.s_free, (gs - 1) & 1, bars, lim, 16)) return false;
       tc_fence_after();
-      const uint32_t kbase = sK + ks * TILE_BYTES;
+      const uint32_t kbase = sKV + (2 * ks) * TILE_BYTES;
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -332,33 +327,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  IDESC_QK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars.s_full);
-        tc_commit(&bars.k_empty[ks]);
       }
       __syncwarp();
       return true;
     };
-    // O_h += P_h V_h for both halves of tile gp
+    // O_h += P_h V_h for both halves of tile gp (its V arrived with its K)
     auto issue_pv = [&](uint32_t gp, bool first) -> bool {
       const int pb = gp & 1;
-      const int vs = gp % VST;
-      if (!wait_warp(&bars.v_full[vs], (gp / VST) & 1, bars, lim, 13)) return false;
+      const int ks = gp % KVST;
       if (first && item_local > 0 && !wait_warp(&bars.o_free, (item_local - 1) & 1, bars, lim, 14)) return false;
-      const uint32_t vbase = sV + vs * TILE_BYTES;
+      if (!wait_warp(&bars.p_full[pb], (gp >> 1) & 1, bars, lim, 12)) return false;
+      tc_fence_after();
+      const uint32_t vbase = sKV + (2 * ks + 1) * TILE_BYTES;
+      if (leader) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (!wait_warp(&bars.p_full[pb][h], (gp >> 1) & 1, bars, lim, 12)) return false;
-        tc_fence_after();
-        if (leader) {
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + TM_O + h * 128, tmem + TM_P + pb * 64 + h * 32 + kk * 8,
                    smem_desc_sw128(vbase + h * 8192 + kk * 2048, HALF_BYTES, 1024), IDESC_PV,
                    (first && kk == 0) ? 0u : 1u);
         }
-        __syncwarp();
-      }
-      if (leader) {
-        tc_commit(&bars.v_empty[vs]);
+        tc_commit(&bars.kv_empty[ks]);
         tc_commit(&bars.pv_done[pb]);
       }
       __syncwarp();
@@ -544,17 +534,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[pb][half]);
+        if (lane == 0) mbar_arrive(&bars.p_full[pb]);
       }
       if (!ok) break;
       // epilogue: merge the two halves' softmax states, write this half's 64
       // output columns: out = (O_0 e_0 + O_1 e_1) / (l_0 e_0 + l_1 e_1),
       // e_h = 2^(m_h - max(m_0, m_1))
-      // (double-buffered by item: a half may finish the next item's key loop
-      // before its partner has read this item's state)
-      const int xb = item_local & 1;
-      bars.xm[xb][half][row] = m_used;
-      bars.xl[xb][half][row] = l;
+      // (one buffer: a half may finish the next item's key loop before its
+      // partner has read this item's state, so writing waits for both reads)
+      if (item_local > 0 && !(ok = wait_warp(&bars.xread, (item_local - 1) & 1, bars, lim, 27))) break;
+      bars.xm[half][row] = m_used;
+      bars.xl[half][row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.xstate);
       if (!(ok = wait_warp(&bars.o_full, item_local & 1, bars, lim, 24))) break;
@@ -569,11 +559,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.o_free);
       if (!(ok = wait_warp(&bars.xstate, item_local & 1, bars, lim, 26))) break;
-      const float m0 = bars.xm[xb][0][row], m1 = bars.xm[xb][1][row];
+      const float m0 = bars.xm[0][row], m1 = bars.xm[1][row];
       const float mm = fmaxf(m0, m1);
       const float e0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
       const float e1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
-      const float inv = 1.0f / (bars.xl[xb][0][row] * e0 + bars.xl[xb][1][row] * e1);
+      const float inv = 1.0f / (bars.xl[0][row] * e0 + bars.xl[1][row] * e1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.xread);
       const float w0 = e0 * inv, w1 = e1 * inv;
       if (row < n_rows) {
 #pragma unroll
