@@ -37,6 +37,31 @@ UNIT = "TFLOP/s (dense-equivalent)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def kernel_source_digest() -> str:
+    """sha256 over the attention kernel's sources (the profile's counters are
+    only reported while the kernel is unchanged since they were taken)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("attn_tc.cu", "sm100.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "video_diffusion_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload_key: str):
+    """DRAM bytes per attention launch from the committed ncu summary of this
+    workload, or None if there is none or the kernel changed since."""
+    p = os.path.join(ROOT, "profiles", f"attn_tc_kernel__{workload_key}_dram.md")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        line = line.strip()
+        if line.startswith("{") and "dram_bytes_per_launch" in line:
+            rec = json.loads(line)
+            if rec.get("kernel_source_sha256") == kernel_source_digest():
+                return float(rec["dram_bytes_per_launch"])
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -69,9 +94,10 @@ def executed_flops(sel: np.ndarray, L: int, B: int, d: int) -> dict:
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms during the timed region."""
+    """nvidia-smi samples every 100 ms; only those taken between mark_start()
+    and mark_end() (the timed region) are summarised."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -79,6 +105,7 @@ class ClockSampler:
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
@@ -86,14 +113,22 @@ class ClockSampler:
             os.close(fd)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(1.0)  # let the sampler start before the timed region
         except Exception:
             self.proc = None
         return self
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.2)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -102,6 +137,7 @@ class ClockSampler:
             self.fh.close()
 
     def summary(self):
+        import datetime as _dt
         if self.proc is None or not self.path or not os.path.exists(self.path):
             return None
         rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
@@ -110,14 +146,17 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             r = [x.strip() for x in r]
-            if len(r) < 9:
+            if len(r) < 10:
                 continue
             try:
-                sm.append(float(r[1]))
-                smax.append(float(r[2]))
+                ts = _dt.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if self.t0 is not None and not (self.t0 - 0.05 <= ts <= (self.t1 or ts) + 0.05):
+                    continue
+                sm.append(float(r[2]))
+                smax.append(float(r[3]))
             except ValueError:
                 continue
-            for name, val in zip(names, r[5:9]):
+            for name, val in zip(names, r[6:10]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
@@ -222,20 +261,75 @@ def aggregate_value(world: int, flops_per_call: float, ms_per_call: float) -> fl
     return world * flops_per_call / (ms_per_call * 1e-3) / 1e12
 
 
+# ----------------------------------------------------------------------------- beta sweep
+
+def sweep_beta(args):
+    """Per beta: selected fraction, ms per call, dense-equivalent and executed
+    TFLOP/s, speedup over the same kernel at beta = -inf, and the error of
+    the output against that dense output."""
+    from video_diffusion_b200 import api
+    from video_diffusion_b200 import inputs as I
+    wl = I.WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    Q, K, V = I.make_workload(wl, device=dev)
+    peak = float(load_peaks()["bf16_tflops"])
+
+    def timed(beta, out):
+        for _ in range(args.warmup):
+            api.forward(Q, K, V, beta, wl.block, out=out)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            api.forward(Q, K, V, beta, wl.block, out=out)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    dense = torch.empty_like(Q)
+    dense_ms = timed(-math.inf, dense)
+    dref = dense.float()
+    for tok in args.sweep_beta.split(","):
+        beta = float(tok)
+        out = torch.empty_like(Q)
+        ms = dense_ms if beta == -math.inf else timed(beta, out)
+        if beta == -math.inf:
+            out = dense
+        counts, sel = api.stats(Q, K, beta, wl.block, with_mask=True)
+        work = executed_flops(sel.cpu().numpy(), wl.L, wl.block, wl.d)
+        diff = out.float() - dref
+        line = {"workload": wl.name, "beta": beta, "selected_fraction": work["selected_fraction"],
+                "gaussian_fraction": 0.5 * math.erfc(beta / math.sqrt(2)) if math.isfinite(beta) else
+                (1.0 if beta < 0 else 0.0),
+                "ms_per_call": ms, "dense_equiv_tflops": wl.dense_flops() / (ms * 1e-3) / 1e12,
+                "executed_tflops": work["total"] / (ms * 1e-3) / 1e12,
+                "pct_bf16_peak": 100 * work["total"] / (ms * 1e-3) / 1e12 / peak,
+                "speedup_vs_dense": dense_ms / ms, "target_speedup": 1.0 / (work["selected_fraction"] + 0.15),
+                "rel_l2_vs_dense": float(diff.norm() / dref.norm()), "max_abs_vs_dense": float(diff.abs().max())}
+        print(json.dumps(line), flush=True)
+        del out, sel, counts, diff
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan-720p")
     ap.add_argument("--beta", type=float, default=1.04)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep-beta", default=None,
+                    help="comma-separated betas: print one line per beta (fraction, time, speedup and "
+                         "error against the beta=-inf output) instead of the benchmark line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.sweep_beta:
+        sweep_beta(args)
+        return
 
     from video_diffusion_b200 import inputs as I
     wl = I.WORKLOADS[args.workload]
@@ -279,11 +373,13 @@ def main():
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        clocks.mark_start()
         start.record(stream)
         for s in range(args.steps):
             api.forward_ex(Q, K, V, args.beta, wl.block, out=out, events=evs[s])
         end.record(stream)
         torch.cuda.synchronize()
+        clocks.mark_end()
     barrier()
     total_ms = start.elapsed_time(end)
     ms_step = max_over_ranks(total_ms / args.steps)
@@ -358,7 +454,8 @@ def main():
         "speedup_vs_dense": (dense_ms / ms_step) if dense_ms else None,
         "target_speedup": 1.0 / (work["selected_fraction"] + 0.15),
         "roofline": {"kernel": "attn_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic(f"{args.workload}_beta{args.beta:g}"),
                      "peak_source": f"{peaks['source']} bf16 burst"},
         "cpu_baseline": cpu,
         "e2e": e2e,

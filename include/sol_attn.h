@@ -25,8 +25,9 @@
  *     enqueued on it; no call synchronises the host, except
  *     sol_attn_device_status().
  *   - Scratch memory (pooled tensors, the 1-bit selection mask, the work list;
- *     about 4% of one input tensor) is taken with cudaMallocAsync on `stream`
- *     and released with cudaFreeAsync on the same stream.
+ *     about 4% of one input tensor) is taken stream-ordered on `stream` from a
+ *     memory pool the library creates per device (it keeps freed memory for
+ *     the next call) and released with cudaFreeAsync on the same stream.
  *   - Return value: SOL_OK or a negative sol_status.  Arguments are checked on
  *     the host before anything is enqueued; on an argument error nothing is
  *     enqueued.  Errors of kernels already enqueued surface at the caller's

@@ -1,8 +1,9 @@
 // api.cu -- the C ABI of libsolattn (declared in include/sol_attn.h).
 //
 // Host-side work only: argument checks, scratch carving (one stream-ordered
-// allocation per call), and the launch sequence pool -> route -> order ->
-// attention on the caller's stream.
+// allocation per call from a library-owned memory pool that keeps its memory
+// between calls), and the launch sequence pool -> route -> order -> attention
+// on the caller's stream.
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -71,6 +72,38 @@ size_t carve(const Geometry& g, size_t op_elem, char* base, Scratch* s) {
   return off;
 }
 
+// One stream-ordered pool per device for the per-call scratch.  Its release
+// threshold is unlimited, so memory freed by one call is reused by the next
+// without going back to the driver (the process's default pool is left as
+// the application configured it).
+constexpr int kPoolDevices = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kPoolDevices] = {};
+
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kPoolDevices) return cudaErrorInvalidDevice;
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    if (!g_pool[dev]) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      e = cudaMemPoolCreate(&g_pool[dev], &props);
+      if (e != cudaSuccess) return e;
+      uint64_t keep = ~0ull;
+      e = cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+      if (e != cudaSuccess) return e;
+    }
+    pool = g_pool[dev];
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, st);
+}
+
 int beta_mode_of(float beta) { return std::isinf(beta) ? (beta < 0 ? -1 : 1) : 0; }
 
 uint64_t wait_limit_ns() {
@@ -99,7 +132,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   Scratch s;
   const size_t bytes = carve(g, use_tc ? 2 : 4, nullptr, &s);
   void* base = nullptr;
-  if (cudaMallocAsync(&base, bytes, st) != cudaSuccess) {
+  if (scratch_alloc(&base, bytes, st) != cudaSuccess) {
     cudaGetLastError();
     return SOL_ERR_NO_MEMORY;
   }
@@ -163,7 +196,7 @@ int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask
   Scratch s;
   const size_t bytes = carve(g, 4, nullptr, &s);
   void* base = nullptr;
-  if (cudaMallocAsync(&base, bytes, st) != cudaSuccess) {
+  if (scratch_alloc(&base, bytes, st) != cudaSuccess) {
     cudaGetLastError();
     return SOL_ERR_NO_MEMORY;
   }
@@ -208,7 +241,7 @@ int sol_attn_version(void) { return 100; }
 // allocation (which can block, fail under fragmentation, or take memory meant
 // for activations) as an error.  sol_attn_forward_noalloc serves them with the
 // same kernels as sol_attn_forward, taking its scratch from the fixed array
-// below instead of cudaMallocAsync.
+// below instead of a stream-ordered allocation.
 
 namespace {
 
