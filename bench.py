@@ -274,14 +274,14 @@ def sweep_beta(args):
     Q, K, V = I.make_workload(wl, device=dev)
     peak = float(load_peaks()["bf16_tflops"])
 
-    def timed(beta, out):
+    def timed(beta, out, keep_or_drop=False):
         for _ in range(args.warmup):
-            api.forward(Q, K, V, beta, wl.block, out=out)
+            api.forward_ex(Q, K, V, beta, wl.block, out=out, keep_or_drop=keep_or_drop)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record()
         for _ in range(args.steps):
-            api.forward(Q, K, V, beta, wl.block, out=out)
+            api.forward_ex(Q, K, V, beta, wl.block, out=out, keep_or_drop=keep_or_drop)
         e1.record()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / args.steps
@@ -298,6 +298,12 @@ def sweep_beta(args):
         counts, sel = api.stats(Q, K, beta, wl.block, with_mask=True)
         work = executed_flops(sel.cpu().numpy(), wl.L, wl.block, wl.d)
         diff = out.float() - dref
+        # the same beta with the correction off (keep-or-drop): what Eqs. 9-10 buy
+        kod = torch.empty_like(Q)
+        kod_ms = dense_ms if beta == -math.inf else timed(beta, kod, keep_or_drop=True)
+        if beta == -math.inf:
+            kod = dense
+        kdiff = kod.float() - dref
         line = {"workload": wl.name, "beta": beta, "selected_fraction": work["selected_fraction"],
                 "gaussian_fraction": 0.5 * math.erfc(beta / math.sqrt(2)) if math.isfinite(beta) else
                 (1.0 if beta < 0 else 0.0),
@@ -305,9 +311,11 @@ def sweep_beta(args):
                 "executed_tflops": work["total"] / (ms * 1e-3) / 1e12,
                 "pct_bf16_peak": 100 * work["total"] / (ms * 1e-3) / 1e12 / peak,
                 "speedup_vs_dense": dense_ms / ms, "target_speedup": 1.0 / (work["selected_fraction"] + 0.15),
-                "rel_l2_vs_dense": float(diff.norm() / dref.norm()), "max_abs_vs_dense": float(diff.abs().max())}
+                "rel_l2_vs_dense": float(diff.norm() / dref.norm()), "max_abs_vs_dense": float(diff.abs().max()),
+                "keep_or_drop": {"ms_per_call": kod_ms, "rel_l2_vs_dense": float(kdiff.norm() / dref.norm()),
+                                 "max_abs_vs_dense": float(kdiff.abs().max())}}
         print(json.dumps(line), flush=True)
-        del out, sel, counts, diff
+        del out, sel, counts, diff, kod, kdiff
 
 
 # ----------------------------------------------------------------------------- GPU arm

@@ -52,6 +52,11 @@ typedef enum {
   SOL_ERR_DEVICE_TIMEOUT = -5   /* a kernel gave up on a bounded wait (see sol_attn_device_status) */
 } sol_status;
 
+/* Flags of sol_attn_forward_ex. */
+#define SOL_FLAG_KEEP_OR_DROP 1u  /* correction off: unselected blocks contribute nothing (the
+                                     "ordinary block sparse" baseline the method is contrasted
+                                     with; a query block with no selected block outputs zeros) */
+
 typedef enum {
   SOL_DTYPE_BF16 = 0,           /* bfloat16 inputs and output; fp32 accumulation */
   SOL_DTYPE_F32 = 1             /* float32 inputs and output; fp32 arithmetic */
@@ -95,15 +100,16 @@ int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask
                    float beta, int dtype, void* stream);
 
 /*
- * Extended forward for measurement.  Arguments as sol_attn_forward plus:
+ * Extended forward.  Arguments as sol_attn_forward plus:
  *   dtype  : sol_dtype of q, k, v, out
+ *   flags  : 0, or SOL_FLAG_KEEP_OR_DROP (unknown bits: SOL_ERR_INVALID_ARG)
  *   events : NULL, or 4 cudaEvent_t the library records on `stream`
  *            before pooling, after pooling, after routing and after the
  *            attention kernel (time each stage with cudaEventElapsedTime)
  */
 int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, int dtype,
                         int batch, int heads, int L, int d, int Bq, int Bk,
-                        float beta, void* const* events, void* stream);
+                        float beta, unsigned int flags, void* const* events, void* stream);
 
 /*
  * Reads and clears this device's status word, which a kernel sets when one of
@@ -137,7 +143,7 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
 /* Human-readable name of a sol_status value. */
 const char* sol_attn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 101. */
 int sol_attn_version(void);
 
 #ifdef __cplusplus

@@ -150,7 +150,8 @@ def route_head(Qh, Kh, Bq: int, Bk: int, beta: float) -> dict:
     return dict(qgeom=qg, kgeom=kg, Qbar=Qbar, Kbar=Kbar, s=s, mu=mu, sigma=sigma, tau=tau, sel=sel)
 
 
-def attend_query_block(Qi, Kh, Vh, kgeom: BlockGeometry, Kbar, Vhat, sel_row, scale: float) -> np.ndarray:
+def attend_query_block(Qi, Kh, Vh, kgeom: BlockGeometry, Kbar, Vhat, sel_row, scale: float,
+                       correction: bool = True) -> np.ndarray:
     """Output rows of one query block, Eqs. 9 and 10 as printed.
 
     D_i = sum_{j in U_i} n_j exp(Q_i K-bar_j^T) + sum_{j in S_i} RowSum(exp(Q_i K_j^T))
@@ -159,10 +160,15 @@ def attend_query_block(Qi, Kh, Vh, kgeom: BlockGeometry, Kbar, Vhat, sel_row, sc
 
     Every exponent is shifted by the row maximum m of all exponents taken; the
     shift multiplies D and N by the same factor and cancels in N / D.
+
+    correction=False is the keep-or-drop baseline the pages contrast Sol-Attn
+    with (visual explainer, "Ordinary block sparse": every unselected block
+    contributes zero): only the "Exact" terms remain.  With no block selected
+    D = N = 0; that row's output is read as 0.
     """
     Qi = np.asarray(Qi, np.float64)
     sel_row = np.asarray(sel_row, bool)
-    approx = np.nonzero(~sel_row)[0]
+    approx = np.nonzero(~sel_row)[0] if correction else np.zeros(0, dtype=np.int64)
     exact = np.nonzero(sel_row)[0]
 
     # Approximate terms: one pooled logit per unselected block and row.
@@ -177,6 +183,8 @@ def attend_query_block(Qi, Kh, Vh, kgeom: BlockGeometry, Kbar, Vhat, sel_row, sc
     x = np.concatenate(xs, axis=1) if xs else np.zeros((Qi.shape[0], 0))
     vx = np.concatenate(vs, axis=0) if vs else np.zeros((0, Vh.shape[1]))
 
+    if a.shape[1] + x.shape[1] == 0:
+        return np.zeros((Qi.shape[0], Vh.shape[1]))
     m = np.max(np.concatenate([a, x], axis=1), axis=1, keepdims=True)
     ea = np.exp(a - m)
     ex = np.exp(x - m)
@@ -186,7 +194,8 @@ def attend_query_block(Qi, Kh, Vh, kgeom: BlockGeometry, Kbar, Vhat, sel_row, sc
     return N / D[:, None]
 
 
-def forward_head(Qh, Kh, Vh, Bq: int, Bk: int, beta: float, sel=None, query_blocks=None):
+def forward_head(Qh, Kh, Vh, Bq: int, Bk: int, beta: float, sel=None, query_blocks=None,
+                 correction: bool = True):
     """One (batch, head): route (or take ``sel`` as given) and attend.
 
     Returns (out [L, d] with NaN in rows of blocks not requested, route dict).
@@ -212,19 +221,21 @@ def forward_head(Qh, Kh, Vh, Bq: int, Bk: int, beta: float, sel=None, query_bloc
     blocks = range(qg.n) if query_blocks is None else query_blocks
     for i in blocks:
         s0, n = int(qg.starts[i]), int(qg.counts[i])
-        out[s0:s0 + n] = attend_query_block(Qh[s0:s0 + n], Kh, Vh, kg, r["Kbar"], Vhat, r["sel_used"][i], scale)
+        out[s0:s0 + n] = attend_query_block(Qh[s0:s0 + n], Kh, Vh, kg, r["Kbar"], Vhat, r["sel_used"][i], scale,
+                                            correction)
     return out, r
 
 
-def forward(Q, K, V, Bq: int, Bk: int, beta: float) -> np.ndarray:
-    """Full forward over [batch, heads, L, d] inputs; float64 output."""
+def forward(Q, K, V, Bq: int, Bk: int, beta: float, correction: bool = True) -> np.ndarray:
+    """Full forward over [batch, heads, L, d] inputs; float64 output
+    (correction=False: the keep-or-drop baseline)."""
     Q = np.asarray(Q, np.float64)
     K = np.asarray(K, np.float64)
     V = np.asarray(V, np.float64)
     out = np.empty_like(Q)
     for b in range(Q.shape[0]):
         for h in range(Q.shape[1]):
-            out[b, h], _ = forward_head(Q[b, h], K[b, h], V[b, h], Bq, Bk, beta)
+            out[b, h], _ = forward_head(Q[b, h], K[b, h], V[b, h], Bq, Bk, beta, correction=correction)
     return out
 
 

@@ -39,7 +39,7 @@ def test_status_strings_and_version(L):
     assert api.status_string(-1) == "SOL_ERR_INVALID_ARG"
     assert api.status_string(-5) == "SOL_ERR_DEVICE_TIMEOUT"
     assert api.status_string(7) == "SOL_ERR_UNKNOWN"
-    assert api.version() == 100
+    assert api.version() == 101
 
 
 # Argument checks run on the host before any CUDA call, so fake device
@@ -68,7 +68,8 @@ def test_stats_and_ex_reject_bad_arguments(L):
     assert L.sol_attn_stats(FAKE, FAKE, None, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, None) == -1
     assert L.sol_attn_stats(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 128, f(1.0), 9, None) == -1
     assert L.sol_attn_stats(FAKE, FAKE, FAKE, None, 1, 1, 256, 100, 128, 128, f(1.0), 0, None) == -2
-    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 5, 1, 1, 256, 128, 128, 128, f(1.0), None, None) == -1
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 5, 1, 1, 256, 128, 128, 128, f(1.0), 0, None, None) == -1
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 128, 128, f(1.0), 6, None, None) == -1
     assert L.sol_attn_forward_f32(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 64, 64, f(math.nan), None) == -1
 
 

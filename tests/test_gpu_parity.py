@@ -169,3 +169,38 @@ def test_video_workloads(name, beta):
     if beta == 1.04:
         frac = sel.mean()
         assert 0.05 < frac < 0.30, frac
+
+
+# ------------------------------------------------------------------ keep-or-drop (correction off)
+
+def check_keep_or_drop(Q, K, V, block, beta):
+    out = torch.full_like(Q, float("nan"))
+    api.forward_ex(Q, K, V, beta, block, out=out, keep_or_drop=True)
+    counts, sel = api.stats(Q, K, beta, block, with_mask=True)
+    torch.cuda.synchronize()
+    sel = sel.cpu().numpy()
+    counts = counts.cpu().numpy()
+    gpu_rows, ref_rows = [], []
+    for b in range(Q.shape[0]):
+        for h in range(Q.shape[1]):
+            r = O.route_head(P.head_np(Q, b, h), P.head_np(K, b, h), block, block, beta)
+            P.compare_selection(r, sel[b, h], counts[b, h])
+            ref, _ = O.forward_head(P.head_np(Q, b, h), P.head_np(K, b, h), P.head_np(V, b, h), block, block,
+                                    beta, sel=sel[b, h], correction=False)
+            ref_rows.append(ref)
+            gpu_rows.append(out[b, h].double().cpu().numpy())
+    assert not torch.isnan(out).any()
+    return P.check_close(np.concatenate(gpu_rows), np.concatenate(ref_rows), Q.dtype, f"keep-or-drop beta={beta}")
+
+
+@pytest.mark.parametrize("beta", [-INF, 0.5, 1.04, 2.0, INF])
+def test_keep_or_drop_bf16(beta):
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=8, device="cuda")  # L = 1000, ragged tail
+    check_keep_or_drop(Q, K, V, 128, beta)
+
+
+@pytest.mark.parametrize("beta", [0.5, 1.04, INF])
+def test_keep_or_drop_fp32(beta):
+    wl = I.WORKLOADS["tiny-fp32"]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    check_keep_or_drop(Q, K, V, wl.block, beta)

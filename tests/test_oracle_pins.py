@@ -267,3 +267,33 @@ def test_stats_counts():
     assert np.all(c_all == 5)
     c_none, _ = O.stats(Q, K, 32, 32, math.inf)
     assert np.all(c_none == 0)
+
+
+# ---------------------------------------------------------------- keep-or-drop baseline (correction off)
+
+def test_keep_or_drop_all_selected_is_dense():
+    Q, K, V = rng_qkv(14, 100, 16)
+    out, _ = O.forward_head(Q[0, 0], K[0, 0], V[0, 0], 16, 16, -math.inf, correction=False)
+    np.testing.assert_allclose(out, O.dense_attention(Q[0, 0], K[0, 0], V[0, 0]), rtol=1e-11, atol=1e-12)
+
+
+def test_keep_or_drop_is_attention_over_selected_tokens_only():
+    """Unselected blocks contribute zero: each query block attends (library
+    SDPA) to the tokens of its selected blocks alone; nothing selected -> 0."""
+    Q, K, V = rng_qkv(15, 90, 8)  # blocks of 16: 5 full + 10 tokens
+    Qh, Kh, Vh = Q[0, 0], K[0, 0], V[0, 0]
+    out, r = O.forward_head(Qh, Kh, Vh, 16, 16, 0.8, correction=False)
+    geom = r["kgeom"]
+    for i in range(r["qgeom"].n):
+        s0, n = int(r["qgeom"].starts[i]), int(r["qgeom"].counts[i])
+        keys = np.concatenate([np.arange(geom.starts[j], geom.starts[j] + geom.counts[j])
+                               for j in np.nonzero(r["sel"][i])[0]] or [np.zeros(0, dtype=np.int64)])
+        if keys.size == 0:
+            np.testing.assert_array_equal(out[s0:s0 + n], 0.0)
+            continue
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Qh[s0:s0 + n])[None], torch.from_numpy(Kh[keys])[None],
+            torch.from_numpy(Vh[keys])[None]).numpy()[0]
+        np.testing.assert_allclose(out[s0:s0 + n], ref, rtol=1e-11, atol=1e-12)
+    out_inf, r_inf = O.forward_head(Qh, Kh, Vh, 16, 16, math.inf, correction=False)
+    assert r_inf["sel"].sum() == 0 and np.all(out_inf == 0.0)

@@ -20,6 +20,7 @@ SOL_OK = 0
 STATUS = {0: "SOL_OK", -1: "SOL_ERR_INVALID_ARG", -2: "SOL_ERR_UNSUPPORTED", -3: "SOL_ERR_CUDA",
           -4: "SOL_ERR_NO_MEMORY", -5: "SOL_ERR_DEVICE_TIMEOUT"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
+FLAG_KEEP_OR_DROP = 1  # correction off: unselected blocks contribute nothing
 
 EXPORTS = ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
            "sol_attn_device_status", "sol_attn_status_string", "sol_attn_version")
@@ -41,14 +42,16 @@ def lib() -> ctypes.CDLL:
         vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.sol_attn_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.sol_attn_forward_f32.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
-        L.sol_attn_forward_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, vp, vp]
+        L.sol_attn_forward_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, ctypes.c_uint,
+                                          vp, vp]
+        L.sol_attn_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.sol_attn_stats.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
         L.sol_attn_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         L.sol_attn_status_string.argtypes = [i32]
         L.sol_attn_status_string.restype = ctypes.c_char_p
         L.sol_attn_version.argtypes = []
         for name in ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
-                     "sol_attn_device_status", "sol_attn_version"):
+                     "sol_attn_device_status", "sol_attn_version", "sol_attn_forward_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -97,10 +100,13 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, bloc
     return out
 
 
-def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, stream=None) -> torch.Tensor:
+def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, stream=None,
+               keep_or_drop: bool = False) -> torch.Tensor:
     """forward() that also records up to four torch.cuda.Event objects: before
     pooling, after pooling, after routing, after the attention kernel.  The
-    events must exist already (torch creates them on their first record())."""
+    events must exist already (torch creates them on their first record()).
+    keep_or_drop=True switches the correction off (unselected blocks
+    contribute nothing; rows with no selected block give 0)."""
     b, h, L, d = _shape(q, k, v)
     if out is None:
         out = torch.empty_like(q)
@@ -113,7 +119,8 @@ def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, st
                 raise ValueError("event not created yet: record it once before passing it")
         ev = ctypes.cast(arr, ctypes.c_void_p)
     rc = lib().sol_attn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
-                                   b, h, L, d, block, block, float(beta), ev, _stream_handle(stream))
+                                   b, h, L, d, block, block, float(beta),
+                                   FLAG_KEEP_OR_DROP if keep_or_drop else 0, ev, _stream_handle(stream))
     _check("sol_attn_forward_ex", rc)
     return out
 

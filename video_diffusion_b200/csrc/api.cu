@@ -122,8 +122,10 @@ int record(void* const* events, int i, cudaStream_t st) {
 }
 
 int forward_impl(const void* q, const void* k, const void* v, void* out, int dtype, int batch, int heads, int L,
-                 int d, int Bq, int Bk, float beta, void* const* events, cudaStream_t st) {
+                 int d, int Bq, int Bk, float beta, unsigned flags, void* const* events, cudaStream_t st) {
   if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
+  if (flags & ~SOL_FLAG_KEEP_OR_DROP) return SOL_ERR_INVALID_ARG;
+  const int correction = (flags & SOL_FLAG_KEEP_OR_DROP) ? 0 : 1;
   Geometry g;
   int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
   if (rc != SOL_OK) return rc;
@@ -143,7 +145,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   e = sol::launch_pool(in_dtype, op_dtype, q, k, v, g, s, st);
   if (e != cudaSuccess) goto done;
   if ((rc = record(events, 1, st)) != SOL_OK) goto done;
-  e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, st);
+  e = sol::launch_route(g, s, beta, beta_mode_of(beta), correction, st);
   if (e != cudaSuccess) goto done;
   e = sol::launch_order(g, s, st);
   if (e != cudaSuccess) goto done;
@@ -151,9 +153,9 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   if (use_tc) {
     e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) goto done;
-    e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns());
+    e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), correction);
   } else {
-    e = sol::launch_attn_simt(in_dtype, q, k, v, out, g, s, st);
+    e = sol::launch_attn_simt(in_dtype, q, k, v, out, g, s, st, correction);
   }
   if (e != cudaSuccess) goto done;
   rc = record(events, 3, st);
@@ -169,19 +171,20 @@ extern "C" {
 
 int sol_attn_forward(const void* q, const void* k, const void* v, void* out, int batch, int heads, int L, int d,
                      int Bq, int Bk, float beta, void* stream) {
-  return forward_impl(q, k, v, out, SOL_DTYPE_BF16, batch, heads, L, d, Bq, Bk, beta, nullptr,
+  return forward_impl(q, k, v, out, SOL_DTYPE_BF16, batch, heads, L, d, Bq, Bk, beta, 0u, nullptr,
                       static_cast<cudaStream_t>(stream));
 }
 
 int sol_attn_forward_f32(const float* q, const float* k, const float* v, float* out, int batch, int heads, int L,
                          int d, int Bq, int Bk, float beta, void* stream) {
-  return forward_impl(q, k, v, out, SOL_DTYPE_F32, batch, heads, L, d, Bq, Bk, beta, nullptr,
+  return forward_impl(q, k, v, out, SOL_DTYPE_F32, batch, heads, L, d, Bq, Bk, beta, 0u, nullptr,
                       static_cast<cudaStream_t>(stream));
 }
 
 int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, int dtype, int batch, int heads,
-                        int L, int d, int Bq, int Bk, float beta, void* const* events, void* stream) {
-  return forward_impl(q, k, v, out, dtype, batch, heads, L, d, Bq, Bk, beta, events,
+                        int L, int d, int Bq, int Bk, float beta, unsigned int flags, void* const* events,
+                        void* stream) {
+  return forward_impl(q, k, v, out, dtype, batch, heads, L, d, Bq, Bk, beta, flags, events,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -229,7 +232,7 @@ const char* sol_attn_status_string(int status) {
   }
 }
 
-int sol_attn_version(void) { return 100; }
+int sol_attn_version(void) { return 101; }
 
 }  // extern "C"
 
@@ -298,9 +301,9 @@ extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void
   if (e == cudaSuccess) e = sol::launch_order(g, s, st);
   if (use_tc) {
     if (e == cudaSuccess) e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
-    if (e == cudaSuccess) e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns());
+    if (e == cudaSuccess) e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), 1);
   } else if (e == cudaSuccess) {
-    e = sol::launch_attn_simt(0, q, k, v, out, g, s, st);
+    e = sol::launch_attn_simt(0, q, k, v, out, g, s, st, 1);
   }
   return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
 }

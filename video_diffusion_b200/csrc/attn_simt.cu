@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(B) attn_simt_kernel(const T* __restrict__ q, c
     }
   }
   if (r < n_rows) {
-    const float inv = 1.0f / l;
+    const float inv = l > 0.f ? 1.0f / l : 0.f;  // nothing attended (keep-or-drop, no block selected): 0
     T* o = out + head + (size_t)(qi * B + r) * D;
 #pragma unroll
     for (int dd = 0; dd < D; ++dd) st_f(o + dd, acc[dd] * inv);
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(B) attn_simt_kernel(const T* __restrict__ q, c
 
 template <typename T>
 cudaError_t dispatch(const void* q, const void* k, const void* v, void* out, const Geometry& g, const Scratch& s,
-                     cudaStream_t st) {
+                     cudaStream_t st, int correction) {
   const float scale = 1.0f / sqrtf((float)g.d);
 #define SOL_SIMT_CASE(D_, B_)                                                                                   \
   if (g.d == D_ && g.B == B_) {                                                                                 \
@@ -147,7 +147,7 @@ cudaError_t dispatch(const void* q, const void* k, const void* v, void* out, con
     if (e != cudaSuccess) return e;                                                                             \
     attn_simt_kernel<T, D_, B_><<<g.nitems, B_, smem, st>>>(                                                    \
         (const T*)q, (const T*)k, (const T*)v, s.kbar, (const float*)s.vbar_op, s.mask, s.order, g.L, g.N, g.W, \
-        g.nchunk, scale, (T*)out);                                                                              \
+        correction ? g.nchunk : 0, scale, (T*)out);                                                                              \
     return cudaGetLastError();                                                                                  \
   }
   SOL_SIMT_CASE(64, 64)
@@ -162,9 +162,9 @@ cudaError_t dispatch(const void* q, const void* k, const void* v, void* out, con
 
 // dtype: 0 = bf16, 1 = fp32.  K-bar (fp32) and V-bar (fp32) come from the pool kernel.
 cudaError_t launch_attn_simt(int dtype, const void* q, const void* k, const void* v, void* out,
-                             const Geometry& g, const Scratch& s, cudaStream_t st) {
-  if (dtype == 1) return dispatch<float>(q, k, v, out, g, s, st);
-  return dispatch<__nv_bfloat16>(q, k, v, out, g, s, st);
+                             const Geometry& g, const Scratch& s, cudaStream_t st, int correction) {
+  if (dtype == 1) return dispatch<float>(q, k, v, out, g, s, st, correction);
+  return dispatch<__nv_bfloat16>(q, k, v, out, g, s, st, correction);
 }
 
 }  // namespace sol

@@ -81,6 +81,7 @@ struct Params {
   int32_t* work_counter;
   __nv_bfloat16* out;
   uint64_t wait_limit_ns;
+  int chunks;           // pooled-key chunks walked per item: nchunk, or 0 without the correction
 };
 
 struct Bars {
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       ++q_uses;
       TileIter ti;
-      ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.nchunk);
+      ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.chunks);
       for (int n = 0; n < T; ++n) {
         int kind = 0, tidx = 0;
         ti.next(kind, tidx);
@@ -419,7 +420,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         continue;
       }
       TileIter ti;
-      ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.nchunk);
+      ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.chunks);
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < T; ++n) {
         int kind = 0, tidx = 0;
@@ -632,7 +633,7 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int planes) {
 }  // namespace
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
-                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns) {
+                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction) {
   CUtensorMap mQ, mK, mV, mKb, mVb;
   if (!make_map(&mQ, q, g.L, g.bH) || !make_map(&mK, k, g.L, g.bH) || !make_map(&mV, v, g.L, g.bH) ||
       !make_map(&mKb, s.kbar_op, g.N, g.bH) || !make_map(&mVb, s.vbar_op, g.N, g.bH))
@@ -645,6 +646,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.mask = s.mask; p.tiles = s.tiles; p.order = s.order; p.work_counter = s.work_counter;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.wait_limit_ns = wait_limit_ns;
+  p.chunks = correction ? g.nchunk : 0;
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

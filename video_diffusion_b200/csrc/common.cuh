@@ -45,10 +45,11 @@ cudaError_t launch_route(const Geometry& g, const Scratch& s, float beta, int be
 cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st);
 
 // Attention launches.
+// correction = 0: keep-or-drop (pooled-key tiles skipped, empty rows give 0).
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
-                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns);
+                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction);
 cudaError_t launch_attn_simt(int dtype, const void* q, const void* k, const void* v, void* out,
-                             const Geometry& g, const Scratch& s, cudaStream_t st);
+                             const Geometry& g, const Scratch& s, cudaStream_t st, int correction);
 cudaError_t read_device_status(cudaStream_t st, int32_t* word);
 
 }  // namespace sol
