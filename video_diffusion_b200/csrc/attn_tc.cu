@@ -65,10 +65,13 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA;
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_P = 384;  // O_h at TM_O + 128 h
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
-// One column pair in POLY_PAIR_PERIOD takes the FMA-pipe polynomial exp2
-// instead of the MUFU ex2 unit (16 of a thread's 64 columns per tile): per
-// tile the MUFU unit, not the FMA pipe, is the tighter of the two.
-constexpr int POLY_PAIR_PERIOD = 4;
+// Column pairs p with (p % 8) in {2, 5, 7} (3 of 8, 24 of a thread's 64
+// columns per tile) take the FMA-pipe polynomial exp2 instead of the MUFU
+// ex2 unit: with 3/8 on the polynomial the MUFU unit and the issue slots of
+// the two softmax warps sharing a scheduler are about equally busy.
+__host__ __device__ constexpr bool poly_pair(int pair) {
+  return (pair & 7) == 2 || (pair & 7) == 5 || (pair & 7) == 7;
+}
 
 struct Params {
   int bH, L, N, W, nchunk, nitems, n_last;
@@ -155,7 +158,9 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Bars& 
 // 2^f from a cubic fitted here to 2^f on [-1/2, 1/2] (least squares with
 // Lawson reweighting toward minimax relative error, max 7.5e-5), then j is
 // added to the exponent field.  Inputs below -125 (where the exponent field
-// would underflow) give exactly 0, as does -inf.
+// would underflow, -inf included) give 2^-125, about 2.4e-38: against row
+// sums of at least 1 that is below float precision, so no select is spent on
+// returning an exact 0.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 xc = make_float2(fmaxf(x.x, -125.0f), fmaxf(x.y, -125.0f));
   const float shifter = 12582912.0f;  // 1.5 * 2^23: xc + shifter rounds xc to an integer in the low bits
@@ -166,9 +171,8 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   p = fma2(p, f, make_float2(0.69326109f, 0.69326109f));
   p = fma2(p, f, make_float2(0.99992806f, 0.99992806f));
   // the low bits of t hold j; shifting them into the exponent field adds j to p's exponent
-  const float r0 = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
-  return make_float2(x.x < -125.0f ? 0.0f : r0, x.y < -125.0f ? 0.0f : r1);
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Max of 64 values with three-input max instructions.
@@ -504,7 +508,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int c = 0; c < 64; c += 2) {
           const float2 a = fma2(make_float2(x[c], x[c + 1]), sl2v, negv);
           float2 e;
-          if (((c >> 1) % POLY_PAIR_PERIOD) == POLY_PAIR_PERIOD - 1) {
+          if (poly_pair(c >> 1)) {
             e = exp2_poly2(a);
           } else {
             e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
@@ -514,8 +518,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         const float2 s2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
         l += s2.x + s2.y;
-        // P buffer pb was read by the PV of tile gs - 2
-        if (gs >= 2 && !(ok = wait_warp(&bars.pv_done[pb], ((gs - 2) >> 1) & 1, bars, lim, 22))) break;
+        // P buffer pb was last read by the PV of tile gs - 2; no wait is needed:
+        // the MMA thread issued that PV before S of tile gs, and the s_full
+        // commit it made after S fires only when all its earlier MMAs are done
         tmem_st32(tmem + lane_off + TM_P + pb * 64 + half * 32, pk);
         if (n > 0 && __any_sync(0xffffffffu, need)) {
           // O_h must hold every PV up to tile gs - 1 before it is rescaled
