@@ -30,6 +30,8 @@ from .sol_attn import (  # noqa: F401
     proxy_scores,
     row_moments,
     eq5_moments,
+    diagonal_sigma,
+    MOMENTS,
     threshold,
     select_blocks,
     route_head,

@@ -116,6 +116,29 @@ def eq5_moments(Qbar: np.ndarray, Kbar: np.ndarray, scale: float) -> tuple[np.nd
     return mu, np.sqrt(np.maximum(var, 0.0))
 
 
+def diagonal_sigma(Qbar: np.ndarray, Kbar: np.ndarray, scale: float) -> np.ndarray:
+    """The cheaper "diagonal estimator" of sigma_i that the Sol-Attn visual
+    explainer names beside Eq. 5 (its formula is not printed there).  Reading:
+    the d x d centred second moment of the pooled keys,
+    C = (1/N) sum_j (K-bar_j - k)^T (K-bar_j - k) with k the mean pooled key,
+    is replaced by its diagonal, so that
+
+        sigma_i^2 ~ scale^2 sum_c Q-bar_{i,c}^2 Var_j(K-bar_{j,c})
+
+    (population variance over the N key blocks).  It equals the Eq. 5 sigma
+    whenever the pooled-key channels are uncorrelated over the blocks, and
+    always when Q-bar_i has one non-zero channel."""
+    Qbar = np.asarray(Qbar, np.float64)
+    Kbar = np.asarray(Kbar, np.float64)
+    N = Kbar.shape[0]
+    kmean = Kbar.sum(axis=0) / N
+    var_c = ((Kbar - kmean[None, :]) ** 2).sum(axis=0) / N    # Var_j(K-bar_{j,c}), one per channel
+    return scale * np.sqrt((Qbar * Qbar) @ var_c)
+
+
+MOMENTS = ("eq5", "diagonal")
+
+
 def threshold(mu: np.ndarray, sigma: np.ndarray, beta: float) -> np.ndarray:
     """tau_i = mu_i + beta sigma_i (Eq. 4).  beta = -inf gives tau = -inf and
     beta = +inf gives tau = +inf for every row, also where sigma_i = 0."""
@@ -134,8 +157,13 @@ def select_blocks(s: np.ndarray, tau: np.ndarray) -> np.ndarray:
     return np.asarray(s, np.float64) > np.asarray(tau, np.float64)[:, None]
 
 
-def route_head(Qh, Kh, Bq: int, Bk: int, beta: float) -> dict:
-    """Steps 1-3 for one (batch, head): pooling, proxy scores, Eq. 4 routing."""
+def route_head(Qh, Kh, Bq: int, Bk: int, beta: float, moments: str = "eq5") -> dict:
+    """Steps 1-3 for one (batch, head): pooling, proxy scores, Eq. 4 routing.
+
+    moments="eq5": mu_i and sigma_i of the score row (Eq. 5).
+    moments="diagonal": the same mu_i, sigma_i from ``diagonal_sigma``."""
+    if moments not in MOMENTS:
+        raise ValueError(moments)
     Qh = np.asarray(Qh, np.float64)
     Kh = np.asarray(Kh, np.float64)
     L, d = Qh.shape
@@ -145,6 +173,8 @@ def route_head(Qh, Kh, Bq: int, Bk: int, beta: float) -> dict:
     Kbar = pool_blocks(Kh, kg, "mean")
     s = proxy_scores(Qbar, Kbar, scale)
     mu, sigma = row_moments(s)
+    if moments == "diagonal":
+        sigma = diagonal_sigma(Qbar, Kbar, scale)
     tau = threshold(mu, sigma, beta)
     sel = select_blocks(s, tau)
     return dict(qgeom=qg, kgeom=kg, Qbar=Qbar, Kbar=Kbar, s=s, mu=mu, sigma=sigma, tau=tau, sel=sel)
@@ -195,7 +225,7 @@ def attend_query_block(Qi, Kh, Vh, kgeom: BlockGeometry, Kbar, Vhat, sel_row, sc
 
 
 def forward_head(Qh, Kh, Vh, Bq: int, Bk: int, beta: float, sel=None, query_blocks=None,
-                 correction: bool = True):
+                 correction: bool = True, moments: str = "eq5"):
     """One (batch, head): route (or take ``sel`` as given) and attend.
 
     Returns (out [L, d] with NaN in rows of blocks not requested, route dict).
@@ -208,7 +238,7 @@ def forward_head(Qh, Kh, Vh, Bq: int, Bk: int, beta: float, sel=None, query_bloc
     Vh = np.asarray(Vh, np.float64)
     L, d = Qh.shape
     scale = 1.0 / math.sqrt(d)
-    r = route_head(Qh, Kh, Bq, Bk, beta)
+    r = route_head(Qh, Kh, Bq, Bk, beta, moments)
     if sel is not None:
         sel = np.asarray(sel, bool)
         assert sel.shape == r["sel"].shape
@@ -226,20 +256,21 @@ def forward_head(Qh, Kh, Vh, Bq: int, Bk: int, beta: float, sel=None, query_bloc
     return out, r
 
 
-def forward(Q, K, V, Bq: int, Bk: int, beta: float, correction: bool = True) -> np.ndarray:
+def forward(Q, K, V, Bq: int, Bk: int, beta: float, correction: bool = True, moments: str = "eq5") -> np.ndarray:
     """Full forward over [batch, heads, L, d] inputs; float64 output
-    (correction=False: the keep-or-drop baseline)."""
+    (correction=False: the keep-or-drop baseline; moments: see route_head)."""
     Q = np.asarray(Q, np.float64)
     K = np.asarray(K, np.float64)
     V = np.asarray(V, np.float64)
     out = np.empty_like(Q)
     for b in range(Q.shape[0]):
         for h in range(Q.shape[1]):
-            out[b, h], _ = forward_head(Q[b, h], K[b, h], V[b, h], Bq, Bk, beta, correction=correction)
+            out[b, h], _ = forward_head(Q[b, h], K[b, h], V[b, h], Bq, Bk, beta, correction=correction,
+                                        moments=moments)
     return out
 
 
-def stats(Q, K, Bq: int, Bk: int, beta: float):
+def stats(Q, K, Bq: int, Bk: int, beta: float, moments: str = "eq5"):
     """Selected-block counts |S_i| [b, H, Nq] and the selection [b, H, Nq, Nk]."""
     Q = np.asarray(Q, np.float64)
     K = np.asarray(K, np.float64)
@@ -248,7 +279,7 @@ def stats(Q, K, Bq: int, Bk: int, beta: float):
     for b in range(Q.shape[0]):
         cb, sb = [], []
         for h in range(Q.shape[1]):
-            r = route_head(Q[b, h], K[b, h], Bq, Bk, beta)
+            r = route_head(Q[b, h], K[b, h], Bq, Bk, beta, moments)
             cb.append(r["sel"].sum(axis=1))
             sb.append(r["sel"])
         counts.append(cb)

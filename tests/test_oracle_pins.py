@@ -147,8 +147,9 @@ def test_beta_minus_inf_is_dense_attention_sdpa():
     np.testing.assert_allclose(O.dense_attention(Q, K, V), ref, rtol=1e-11, atol=1e-12)
 
 
+@pytest.mark.parametrize("Bq", (16, 8, 32))
 @pytest.mark.parametrize("beta", BETAS)
-def test_identical_keys_per_block_give_dense_attention(beta):
+def test_identical_keys_per_block_give_dense_attention(beta, Bq):
     """Eqs. 9/10 replace every key of an unselected block by its mean; when the
     keys of each block are identical that is exact, so every beta gives dense
     attention (Q and V still vary token by token)."""
@@ -159,7 +160,7 @@ def test_identical_keys_per_block_give_dense_attention(beta):
     K = np.concatenate([np.repeat(Kblk[j][None], geom.counts[j], 0) for j in range(geom.n)])
     Q = g.standard_normal((L, d)) * 1.5
     V = g.standard_normal((L, d))
-    out, r = O.forward_head(Q, K, V, B, B, beta)
+    out, r = O.forward_head(Q, K, V, Bq, B, beta)
     np.testing.assert_allclose(out, O.dense_attention(Q, K, V), rtol=1e-11, atol=1e-12)
 
 
@@ -205,7 +206,7 @@ def test_key_block_permutation_invariance():
         np.testing.assert_array_equal(r1["sel"][:, full], r2["sel"])
 
 
-def _brute_force_key_replacement(Q, K, V, B, beta):
+def _brute_force_key_replacement(Q, K, V, Bq, Bk, beta):
     """Pure-Python restatement in the derivation's own terms: a query block
     keeps the original keys of its selected blocks and sees every key of an
     unselected block replaced by that block's mean key; values are untouched
@@ -213,13 +214,14 @@ def _brute_force_key_replacement(Q, K, V, B, beta):
     unselected block by its mean)."""
     L, d = len(Q), len(Q[0])
     scale = 1 / math.sqrt(d)
-    nb = (L + B - 1) // B
-    blocks = [list(range(b * B, min(L, b * B + B))) for b in range(nb)]
+    nb = (L + Bk - 1) // Bk
+    blocks = [list(range(b * Bk, min(L, b * Bk + Bk))) for b in range(nb)]
+    qblocks = [list(range(b * Bq, min(L, b * Bq + Bq))) for b in range((L + Bq - 1) // Bq)]
     mean = lambda rows, X: [sum(X[r][c] for r in rows) / len(rows) for c in range(d)]
-    Qb = [mean(bl, Q) for bl in blocks]
+    Qb = [mean(bl, Q) for bl in qblocks]
     Kb = [mean(bl, K) for bl in blocks]
     out = [[0.0] * d for _ in range(L)]
-    for i, qb in enumerate(blocks):
+    for i, qb in enumerate(qblocks):
         s = [scale * sum(Qb[i][c] * Kb[j][c] for c in range(d)) for j in range(nb)]
         mu = sum(s) / nb
         sd = math.sqrt(sum((x - mu) ** 2 for x in s) / nb)
@@ -237,13 +239,14 @@ def _brute_force_key_replacement(Q, K, V, B, beta):
     return out
 
 
+@pytest.mark.parametrize("Bq,Bk", ((4, 4), (3, 5), (6, 4)))  # key blocks 4,4,4,2 / 5,5,4
 @pytest.mark.parametrize("beta", (-math.inf, 0.0, 0.5, 1.04, math.inf))
-def test_bruteforce_key_replacement_tiny(beta):
+def test_bruteforce_key_replacement_tiny(beta, Bq, Bk):
     g = np.random.default_rng(11)
-    L, d, B = 14, 3, 4  # blocks 4, 4, 4, 2
+    L, d = 14, 3
     Q, K, V = g.standard_normal((L, d)) * 2, g.standard_normal((L, d)) * 2, g.standard_normal((L, d))
-    ref = _brute_force_key_replacement(Q.tolist(), K.tolist(), V.tolist(), B, beta)
-    out, _ = O.forward_head(Q, K, V, B, B, beta)
+    ref = _brute_force_key_replacement(Q.tolist(), K.tolist(), V.tolist(), Bq, Bk, beta)
+    out, _ = O.forward_head(Q, K, V, Bq, Bk, beta)
     np.testing.assert_allclose(out, np.array(ref), rtol=1e-12, atol=1e-13)
 
 
@@ -297,3 +300,86 @@ def test_keep_or_drop_is_attention_over_selected_tokens_only():
         np.testing.assert_allclose(out[s0:s0 + n], ref, rtol=1e-11, atol=1e-12)
     out_inf, r_inf = O.forward_head(Qh, Kh, Vh, 16, 16, math.inf, correction=False)
     assert r_inf["sel"].sum() == 0 and np.all(out_inf == 0.0)
+
+
+# ---------------------------------------------------------------- diagonal moment estimator (reading)
+
+def test_diagonal_sigma_hand_example():
+    """Two pooled keys (1, 0) and (3, 2): each channel has population variance 1
+    and the channels are perfectly correlated (covariance 1).  Worked by hand:
+    Q-bar = (1, 1): scores 1 and 5, row sigma 2; the diagonal drops the 2*1*1*1
+    cross term, sigma^2 = 1 + 1 = 2.  Q-bar = (2, -1): scores 2 and 4, row
+    sigma 1; diagonal sigma^2 = 4 * 1 + 1 * 1 = 5."""
+    Kbar = np.array([[1.0, 0.0], [3.0, 2.0]])
+    Qbar = np.array([[1.0, 1.0], [2.0, -1.0]])
+    _, sd_row = O.row_moments(O.proxy_scores(Qbar, Kbar, 1.0))
+    np.testing.assert_allclose(sd_row, [2.0, 1.0], rtol=1e-15)
+    np.testing.assert_allclose(O.diagonal_sigma(Qbar, Kbar, 1.0), [math.sqrt(2.0), math.sqrt(5.0)], rtol=1e-15)
+    np.testing.assert_allclose(O.diagonal_sigma(Qbar, Kbar, 0.5), [math.sqrt(2.0) / 2, math.sqrt(5.0) / 2],
+                               rtol=1e-15)
+
+
+def test_diagonal_sigma_equals_row_sigma_for_single_channel_queries():
+    g = np.random.default_rng(21)
+    Kbar = g.standard_normal((40, 8)) @ g.standard_normal((8, 8)) + 0.7  # correlated channels
+    scale = 1 / math.sqrt(8)
+    Qbar = np.zeros((8, 8))
+    Qbar[np.arange(8), np.arange(8)] = g.standard_normal(8) * 3
+    _, sd_row = O.row_moments(O.proxy_scores(Qbar, Kbar, scale))
+    np.testing.assert_allclose(O.diagonal_sigma(Qbar, Kbar, scale), sd_row, rtol=1e-12)
+
+
+def hadamard(n):
+    H = np.array([[1.0]])
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def test_diagonal_sigma_equals_row_sigma_for_uncorrelated_channels():
+    """Columns 1..d of a Sylvester Hadamard matrix sum to zero and are mutually
+    orthogonal, so pooled keys built from them have a diagonal covariance."""
+    g = np.random.default_rng(22)
+    N, d = 32, 12
+    Kbar = 0.4 + hadamard(N)[:, 1:d + 1] * g.uniform(0.5, 2.0, d)[None, :]
+    Qbar = g.standard_normal((20, d))
+    scale = 1 / math.sqrt(d)
+    _, sd_row = O.row_moments(O.proxy_scores(Qbar, Kbar, scale))
+    np.testing.assert_allclose(O.diagonal_sigma(Qbar, Kbar, scale), sd_row, rtol=1e-12)
+
+
+def test_diagonal_sigma_misses_exactly_the_off_diagonal_covariance():
+    """Row variance - diagonal variance = scale^2 Q-bar (C - diag C) Q-bar^T with
+    C the population covariance of the pooled keys (numpy.cov, bias=True)."""
+    g = np.random.default_rng(23)
+    Kbar = g.standard_normal((50, 6)) @ g.standard_normal((6, 6)) - 0.3
+    Qbar = g.standard_normal((15, 6))
+    scale = 0.37
+    _, sd_row = O.row_moments(O.proxy_scores(Qbar, Kbar, scale))
+    C = np.cov(Kbar.T, bias=True)
+    off = C - np.diag(np.diag(C))
+    gap = scale ** 2 * np.einsum("ic,ce,ie->i", Qbar, off, Qbar)
+    np.testing.assert_allclose(sd_row ** 2 - O.diagonal_sigma(Qbar, Kbar, scale) ** 2, gap, atol=1e-12)
+
+
+def test_diagonal_routing_matches_eq5_routing_when_channels_are_uncorrelated():
+    """Keys constant inside each block with Hadamard-structured block means:
+    both estimators give the same sigma, hence the same selection; on generic
+    keys they differ somewhere."""
+    g = np.random.default_rng(24)
+    N, B, d = 16, 8, 8
+    kb = 0.2 + hadamard(N)[:, 1:d + 1] * g.uniform(0.5, 1.5, d)[None, :]
+    K = np.repeat(kb, B, axis=0)[: N * B - 3]   # ragged tail block keeps the same mean
+    Q = g.standard_normal((K.shape[0], d))
+    for beta in (-math.inf, -0.5, 0.5, 1.04, math.inf):
+        a = O.route_head(Q, K, B, B, beta, "eq5")
+        b = O.route_head(Q, K, B, B, beta, "diagonal")
+        np.testing.assert_allclose(a["sigma"], b["sigma"], rtol=1e-12)
+        assert np.all(np.abs(a["s"] - a["tau"][:, None]) > 1e-9) or not np.isfinite(beta)
+        assert np.array_equal(a["sel"], b["sel"])
+    Kg = g.standard_normal((N * B, d)) @ g.standard_normal((d, d))
+    a = O.route_head(Q[: N * B - 3], Kg[: N * B - 3], B, B, 1.04, "eq5")
+    b = O.route_head(Q[: N * B - 3], Kg[: N * B - 3], B, B, 1.04, "diagonal")
+    assert not np.allclose(a["sigma"], b["sigma"])
+    with pytest.raises(ValueError):
+        O.route_head(Q, K, B, B, 1.0, "full")
