@@ -73,20 +73,27 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- work accounting
 
-def executed_flops(sel: np.ndarray, L: int, B: int, d: int) -> dict:
-    """Algorithmic FLOPs of one call from the selection [b, H, N, N] (bool).
-
-    exact:  4 n_i n_j d for every selected pair (QK^T and PV);
-    approx: 2 n_i N d (token-to-pooled-key scores) + 2 n_i |U_i| d (pooled PV).
-    Padding, masked columns and skipped chunk columns are not counted.
-    """
-    N = sel.shape[-1]
+def block_tokens(L: int, B: int) -> np.ndarray:
+    """Token count of each of the ceil(L / B) blocks."""
+    N = -(-L // B)
     n = np.full(N, B, dtype=np.float64)
     n[-1] = L - (N - 1) * B
-    exact = 4.0 * d * np.einsum("bhij,i,j->", sel.astype(np.float64), n, n)
-    unsel = (~sel).sum(axis=-1).astype(np.float64)  # |U_i|, [b, H, N]
-    rows_with_approx = ((unsel > 0) * n[None, None, :]).sum()
-    approx = 2.0 * d * N * float(rows_with_approx) + 2.0 * d * float((unsel * n[None, None, :]).sum())
+    return n
+
+
+def executed_flops(sel: np.ndarray, L: int, Bq: int, Bk: int, d: int) -> dict:
+    """Algorithmic FLOPs of one call from the selection [b, H, Nq, Nk] (bool).
+
+    exact:  4 n_i n_j d for every selected pair (QK^T and PV);
+    approx: 2 n_i Nk d (token-to-pooled-key scores) + 2 n_i |U_i| d (pooled PV).
+    Padding, masked columns and skipped chunk columns are not counted.
+    """
+    Nk = sel.shape[-1]
+    nq, nk = block_tokens(L, Bq), block_tokens(L, Bk)
+    exact = 4.0 * d * np.einsum("bhij,i,j->", sel.astype(np.float64), nq, nk)
+    unsel = (~sel).sum(axis=-1).astype(np.float64)  # |U_i|, [b, H, Nq]
+    rows_with_approx = ((unsel > 0) * nq[None, None, :]).sum()
+    approx = 2.0 * d * Nk * float(rows_with_approx) + 2.0 * d * float((unsel * nq[None, None, :]).sum())
     return {"exact": float(exact), "approx": float(approx), "total": float(exact + approx),
             "selected_fraction": float(sel.mean())}
 
@@ -167,15 +174,16 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- oracle timing (host)
 
-def oracle_sample_time(wl, beta: float, n_blocks: int = 2, seed: int = 0):
+def oracle_sample_time(wl, beta: float, n_blocks: int = 2, seed: int = 0, block_k=None, moments="eq5"):
     """Times the float64 oracle on one head's pooling + routing and `n_blocks`
     query blocks of attention, and extrapolates to the whole call."""
     from oracle import sol_attn as O
     from video_diffusion_b200 import inputs as I
     Q, K, V = I.make_qkv(wl.grid, 1, wl.d, wl.seed + seed, 1, wl.text_tokens, wl.dtype, "cpu")
     Qh, Kh, Vh = (t[0, 0].double().numpy() for t in (Q, K, V))
+    bq, bk = wl.block, block_k or wl.block
     t0 = time.perf_counter()
-    r = O.route_head(Qh, Kh, wl.block, wl.block, beta)
+    r = O.route_head(Qh, Kh, bq, bk, beta, moments)
     Vhat = O.pool_blocks(Vh, r["kgeom"], "sum")
     t1 = time.perf_counter()
     N = r["qgeom"].n
@@ -205,7 +213,8 @@ def run_reference(args, wl):
         return
     times = []
     for s in range(args.warmup + args.steps):
-        t, cores, sample, frac = oracle_sample_time(wl, args.beta, n_blocks=1, seed=s)
+        t, cores, sample, frac = oracle_sample_time(wl, args.beta, n_blocks=1, seed=s, block_k=args.block_k,
+                                                    moments=moments_of(args))
         if s >= args.warmup:
             times.append(t)
     t = statistics.mean(times)
@@ -222,9 +231,37 @@ def run_reference(args, wl):
 
 
 def config_of(wl, args):
-    return {"workload": wl.name, "beta": args.beta, "batch": wl.batch, "heads": wl.heads, "L": wl.L,
-            "d": wl.d, "block": wl.block, "parallelism": f"replicas x{args.gpus} (independent calls)",
-            "l2": "inputs 2.3 GB per step, larger than the 126 MB L2; no flush"}
+    c = {"workload": wl.name, "beta": args.beta, "batch": wl.batch, "heads": wl.heads, "L": wl.L,
+         "d": wl.d, "block": wl.block, "parallelism": f"replicas x{args.gpus} (independent calls)",
+         "l2": f"inputs {3 * wl.batch * wl.heads * wl.L * wl.d * 2 / 1e9:.2f} GB per step "
+               f"({'larger' if 3 * wl.batch * wl.heads * wl.L * wl.d * 2 > 126e6 else 'smaller'} than the "
+               f"126 MB L2); no flush"}
+    if args.block_k and args.block_k != wl.block:
+        c["block_k"] = args.block_k
+    if args.diagonal_sigma:
+        c["sigma"] = "diagonal estimator"
+    return c
+
+
+def moments_of(args) -> str:
+    return "diagonal" if args.diagonal_sigma else "eq5"
+
+
+def blocks_of(wl, args):
+    return (wl.block, args.block_k or wl.block)
+
+
+def attention_kernel_name(wl, blk) -> str:
+    """The library runs tcgen05 for bf16, d = 128, Bq = 128, Bk in {64, 128}."""
+    tc = wl.dtype == torch.bfloat16 and wl.d == 128 and blk[0] == 128 and blk[1] in (64, 128)
+    return "attn_tc_kernel" if tc else "attn_simt_kernel"
+
+
+def workload_key(wl, args) -> str:
+    key = f"{wl.name}_beta{args.beta:g}"
+    if args.block_k and args.block_k != wl.block:
+        key += f"_bk{args.block_k}"
+    return key
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -270,18 +307,20 @@ def sweep_beta(args):
     from video_diffusion_b200 import api
     from video_diffusion_b200 import inputs as I
     wl = I.WORKLOADS[args.workload]
+    blk = blocks_of(wl, args)
+    diag = bool(args.diagonal_sigma)
     dev = torch.device("cuda", 0)
     Q, K, V = I.make_workload(wl, device=dev)
     peak = float(load_peaks()["bf16_tflops"])
 
     def timed(beta, out, keep_or_drop=False):
         for _ in range(args.warmup):
-            api.forward_ex(Q, K, V, beta, wl.block, out=out, keep_or_drop=keep_or_drop)
+            api.forward_ex(Q, K, V, beta, blk, out=out, keep_or_drop=keep_or_drop, diagonal_sigma=diag)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record()
         for _ in range(args.steps):
-            api.forward_ex(Q, K, V, beta, wl.block, out=out, keep_or_drop=keep_or_drop)
+            api.forward_ex(Q, K, V, beta, blk, out=out, keep_or_drop=keep_or_drop, diagonal_sigma=diag)
         e1.record()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / args.steps
@@ -295,8 +334,8 @@ def sweep_beta(args):
         ms = dense_ms if beta == -math.inf else timed(beta, out)
         if beta == -math.inf:
             out = dense
-        counts, sel = api.stats(Q, K, beta, wl.block, with_mask=True)
-        work = executed_flops(sel.cpu().numpy(), wl.L, wl.block, wl.d)
+        counts, sel = api.stats(Q, K, beta, blk, with_mask=True, diagonal_sigma=diag)
+        work = executed_flops(sel.cpu().numpy(), wl.L, blk[0], blk[1], wl.d)
         diff = out.float() - dref
         # the same beta with the correction off (keep-or-drop): what Eqs. 9-10 buy
         kod = torch.empty_like(Q)
@@ -304,7 +343,8 @@ def sweep_beta(args):
         if beta == -math.inf:
             kod = dense
         kdiff = kod.float() - dref
-        line = {"workload": wl.name, "beta": beta, "selected_fraction": work["selected_fraction"],
+        line = {"workload": wl.name, "block": list(blk), "sigma": moments_of(args), "beta": beta,
+                "selected_fraction": work["selected_fraction"],
                 "gaussian_fraction": 0.5 * math.erfc(beta / math.sqrt(2)) if math.isfinite(beta) else
                 (1.0 if beta < 0 else 0.0),
                 "ms_per_call": ms, "dense_equiv_tflops": wl.dense_flops() / (ms * 1e-3) / 1e12,
@@ -330,6 +370,10 @@ def main():
     ap.add_argument("--beta", type=float, default=1.04)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block-k", type=int, default=None,
+                    help="key block size (default: the workload's block size, the same as the query block)")
+    ap.add_argument("--diagonal-sigma", action="store_true",
+                    help="sigma_i of Eq. 4 from the diagonal moment estimator instead of Eq. 5")
     ap.add_argument("--sweep-beta", default=None,
                     help="comma-separated betas: print one line per beta (fraction, time, speedup and "
                          "error against the beta=-inf output) instead of the benchmark line")
@@ -364,13 +408,15 @@ def main():
     out = torch.empty_like(Q)
     stream = torch.cuda.current_stream()
 
+    blk = blocks_of(wl, args)
+    diag = bool(args.diagonal_sigma)
     # selection statistics (same routing as the forward) for the FLOP count
-    counts, sel = api.stats(Q, K, args.beta, wl.block, with_mask=True)
-    work = executed_flops(sel.cpu().numpy(), wl.L, wl.block, wl.d)
+    counts, sel = api.stats(Q, K, args.beta, blk, with_mask=True, diagonal_sigma=diag)
+    work = executed_flops(sel.cpu().numpy(), wl.L, blk[0], blk[1], wl.d)
     del sel, counts
 
     for _ in range(args.warmup):
-        api.forward(Q, K, V, args.beta, wl.block, out=out)
+        api.forward_ex(Q, K, V, args.beta, blk, out=out, diagonal_sigma=diag)
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -384,7 +430,7 @@ def main():
         clocks.mark_start()
         start.record(stream)
         for s in range(args.steps):
-            api.forward_ex(Q, K, V, args.beta, wl.block, out=out, events=evs[s])
+            api.forward_ex(Q, K, V, args.beta, blk, out=out, events=evs[s], diagonal_sigma=diag)
         end.record(stream)
         torch.cuda.synchronize()
         clocks.mark_end()
@@ -403,11 +449,11 @@ def main():
     dense_ms = None
     if args.beta != -math.inf:
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        api.forward(Q, K, V, -math.inf, wl.block, out=out)
+        api.forward(Q, K, V, -math.inf, blk, out=out)
         torch.cuda.synchronize()
         d0.record(stream)
         for _ in range(2):
-            api.forward(Q, K, V, -math.inf, wl.block, out=out)
+            api.forward(Q, K, V, -math.inf, blk, out=out)
         d1.record(stream)
         torch.cuda.synchronize()
         dense_ms = max_over_ranks(d0.elapsed_time(d1) / 2)
@@ -427,7 +473,7 @@ def main():
             dQ.copy_(hQ, non_blocking=True)
             dK.copy_(hK, non_blocking=True)
             dV.copy_(hV, non_blocking=True)
-            api.forward(dQ, dK, dV, args.beta, wl.block, out=out)
+            api.forward_ex(dQ, dK, dV, args.beta, blk, out=out, diagonal_sigma=diag)
             hO.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -439,7 +485,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, cores, sample, _ = oracle_sample_time(wl, args.beta, n_blocks=2)
+        t, cores, sample, _ = oracle_sample_time(wl, args.beta, n_blocks=2, block_k=args.block_k,
+                                                 moments=moments_of(args))
         cpu = {"value": wl.dense_flops() / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": sample, "extrapolated_s_per_call": t}
 
@@ -461,13 +508,13 @@ def main():
         "dense_ms_per_call": dense_ms,
         "speedup_vs_dense": (dense_ms / ms_step) if dense_ms else None,
         "target_speedup": 1.0 / (work["selected_fraction"] + 0.15),
-        "roofline": {"kernel": "attn_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic(f"{args.workload}_beta{args.beta:g}"),
+        "roofline": {"kernel": attention_kernel_name(wl, blk), "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic(workload_key(wl, args)),
                      "peak_source": f"{peaks['source']} bf16 burst"},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (5 if diag else 4) * args.steps,
         "clocks": clock_summary,
     }
     if rank == 0:

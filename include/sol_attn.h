@@ -5,10 +5,11 @@
  * in one pass", Eqs. 4, 5, 9, 10, 11): for every (batch, head)
  *   1. pool:   Qbar_i = mean of the query rows of block i, Kbar_j = mean of the
  *              key rows of block j, Vhat_j = sum of the value rows of block j
- *              (blocks are contiguous runs of B tokens; the last may be partial,
- *              with n_j < B tokens);
+ *              (blocks are contiguous runs of Bq query / Bk key tokens; the
+ *              last may be partial, key block j holding n_j tokens);
  *   2. score:  s_ij = Qbar_i . Kbar_j / sqrt(d)                      (Eq. 4 legend)
- *   3. route:  mu_i, sigma_i = mean and population std of row s_i.   (Eq. 5)
+ *   3. route:  mu_i, sigma_i = mean and population std of row s_i    (Eq. 5)
+ *              (or sigma_i from the diagonal estimator, see the flags);
  *              tau_i = mu_i + beta * sigma_i; S_i = { j : s_ij > tau_i } (Eq. 4)
  *   4. attend: for every query token q of block i
  *                D = sum_{j in U_i} n_j exp(q.Kbar_j/sqrt d) + sum_{j in S_i} sum_{k in j} exp(q.k/sqrt d)  (Eq. 9)
@@ -52,10 +53,16 @@ typedef enum {
   SOL_ERR_DEVICE_TIMEOUT = -5   /* a kernel gave up on a bounded wait (see sol_attn_device_status) */
 } sol_status;
 
-/* Flags of sol_attn_forward_ex. */
+/* Flags of sol_attn_forward_ex and sol_attn_stats_ex. */
 #define SOL_FLAG_KEEP_OR_DROP 1u  /* correction off: unselected blocks contribute nothing (the
                                      "ordinary block sparse" baseline the method is contrasted
                                      with; a query block with no selected block outputs zeros) */
+#define SOL_FLAG_DIAGONAL_SIGMA 2u /* sigma_i of Eq. 4 from the cheaper diagonal estimator the
+                                     explainer names beside Eq. 5 (formula not printed; read as
+                                     sigma_i^2 = sum_c Qbar_ic^2 Var_j(Kbar_jc) / d, the population
+                                     variance of each pooled-key channel over the key blocks,
+                                     i.e. Eq. 5 with the off-diagonal covariance dropped).
+                                     mu_i is unchanged. */
 
 typedef enum {
   SOL_DTYPE_BF16 = 0,           /* bfloat16 inputs and output; fp32 accumulation */
@@ -63,17 +70,20 @@ typedef enum {
 } sol_dtype;
 
 /*
- * Supported shapes: d in {64, 128}; Bq == Bk in {64, 128}; L >= 1;
- * batch * heads >= 1; batch * heads * L * d < 2^31; beta not NaN.
- * bf16 with d == 128 and B == 128 runs the tensor-core (tcgen05/TMEM/TMA)
- * kernel; every other supported combination runs the CUDA-core kernel.
+ * Supported shapes: d in {64, 128}; Bq in {64, 128} and Bk in {64, 128}
+ * (independently: query blocks of Bq tokens, key blocks of Bk tokens, the
+ * Eq. 9 weight of a key block is its token count); L >= 1; batch * heads >= 1;
+ * batch * heads * L * d < 2^40; ceil(L / Bk) <= 40960; beta not NaN.
+ * Other values return SOL_ERR_UNSUPPORTED.  bf16 with d == Bq == Bk == 128
+ * runs the tensor-core (tcgen05/TMEM/TMA) kernel; every other supported
+ * combination runs the CUDA-core kernel.
  */
 
 /*
  * Sparse attention forward, bf16.
  *   q, k, v : const bf16*  [batch, heads, L, d], device
  *   out     : bf16*        [batch, heads, L, d], device, written fully
- *   Bq, Bk  : query / key block size in tokens (must be equal)
+ *   Bq, Bk  : query / key block size in tokens
  *   beta    : Eq. 4 knob; -INFINITY = dense, +INFINITY = all approximate
  *   stream  : cudaStream_t
  */
@@ -99,10 +109,17 @@ int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask
                    int batch, int heads, int L, int d, int Bq, int Bk,
                    float beta, int dtype, void* stream);
 
+/* sol_attn_stats with flags: 0 or SOL_FLAG_DIAGONAL_SIGMA (any other bit:
+ * SOL_ERR_INVALID_ARG).  sol_attn_stats(...) is sol_attn_stats_ex(..., 0, stream). */
+int sol_attn_stats_ex(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null,
+                      int batch, int heads, int L, int d, int Bq, int Bk,
+                      float beta, int dtype, unsigned int flags, void* stream);
+
 /*
  * Extended forward.  Arguments as sol_attn_forward plus:
  *   dtype  : sol_dtype of q, k, v, out
- *   flags  : 0, or SOL_FLAG_KEEP_OR_DROP (unknown bits: SOL_ERR_INVALID_ARG)
+ *   flags  : 0 or an OR of SOL_FLAG_KEEP_OR_DROP, SOL_FLAG_DIAGONAL_SIGMA
+ *            (unknown bits: SOL_ERR_INVALID_ARG)
  *   events : NULL, or 4 cudaEvent_t the library records on `stream`
  *            before pooling, after pooling, after routing and after the
  *            attention kernel (time each stage with cudaEventElapsedTime)
@@ -143,7 +160,7 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
 /* Human-readable name of a sol_status value. */
 const char* sol_attn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor): 101. */
+/* Library ABI version (major * 100 + minor): 102. */
 int sol_attn_version(void);
 
 #ifdef __cplusplus

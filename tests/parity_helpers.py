@@ -55,16 +55,26 @@ def sample_blocks(N: int, counts_row: np.ndarray, k: int, rng: np.random.Generat
     return sorted(pick)
 
 
-def oracle_rows(Q, K, V, b, h, block, beta, sel, blocks):
+def pair(block) -> tuple[int, int]:
+    """(Bq, Bk) from one block size or a (query, key) pair."""
+    if isinstance(block, (tuple, list)):
+        return int(block[0]), int(block[1])
+    return int(block), int(block)
+
+
+def oracle_rows(Q, K, V, b, h, block, beta, sel, blocks, moments="eq5", correction=True):
     """Oracle output rows of the given query blocks of head (b, h), using the
     selection `sel` (the GPU's, checked against the oracle's beforehand)."""
-    out, _ = O.forward_head(head_np(Q, b, h), head_np(K, b, h), head_np(V, b, h), block, block, beta,
-                            sel=sel, query_blocks=blocks)
+    bq, bk = pair(block)
+    out, _ = O.forward_head(head_np(Q, b, h), head_np(K, b, h), head_np(V, b, h), bq, bk, beta,
+                            sel=sel, query_blocks=blocks, moments=moments, correction=correction)
     return out
 
 
 def rows_of(blocks, block, L):
+    """Token rows of the given query blocks (block: Bq or a (Bq, Bk) pair)."""
+    bq = pair(block)[0]
     idx = []
     for i in blocks:
-        idx.extend(range(i * block, min(L, i * block + block)))
+        idx.extend(range(i * bq, min(L, i * bq + bq)))
     return np.asarray(idx, dtype=np.int64)

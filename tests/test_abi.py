@@ -39,7 +39,7 @@ def test_status_strings_and_version(L):
     assert api.status_string(-1) == "SOL_ERR_INVALID_ARG"
     assert api.status_string(-5) == "SOL_ERR_DEVICE_TIMEOUT"
     assert api.status_string(7) == "SOL_ERR_UNKNOWN"
-    assert api.version() == 101
+    assert api.version() == 102
 
 
 # Argument checks run on the host before any CUDA call, so fake device
@@ -56,8 +56,8 @@ def call_fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, b=1, h=1, n=256, d=128, bq=128, 
     (dict(q=FAKE + 8), -1), (dict(o=FAKE + 2), -1),
     (dict(b=0), -1), (dict(h=0), -1), (dict(n=0), -1), (dict(d=0), -1),
     (dict(beta=float("nan")), -1),
-    (dict(d=96), -2), (dict(d=256), -2), (dict(bq=64, bk=128), -2), (dict(bq=32, bk=32), -2),
-    (dict(bq=256, bk=256), -2),
+    (dict(d=96), -2), (dict(d=256), -2), (dict(bq=96, bk=128), -2), (dict(bq=128, bk=32), -2),
+    (dict(bq=32, bk=32), -2), (dict(bq=256, bk=256), -2), (dict(bq=128, bk=256), -2),
 ])
 def test_forward_rejects_bad_arguments(L, kw, code):
     assert call_fwd(L, **kw) == code
@@ -71,6 +71,13 @@ def test_stats_and_ex_reject_bad_arguments(L):
     assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 5, 1, 1, 256, 128, 128, 128, f(1.0), 0, None, None) == -1
     assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 128, 128, f(1.0), 6, None, None) == -1
     assert L.sol_attn_forward_f32(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 64, 64, f(math.nan), None) == -1
+    # stats_ex takes SOL_FLAG_DIAGONAL_SIGMA only; forward_ex both flags, no other bit
+    assert L.sol_attn_stats_ex(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, 1, None) == -1
+    assert L.sol_attn_stats_ex(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, 4, None) == -1
+    assert L.sol_attn_stats_ex(FAKE, FAKE, None, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, 2, None) == -1
+    assert L.sol_attn_stats_ex(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 96, f(1.0), 0, 2, None) == -2
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 128, 128, f(1.0), 4, None, None) == -1
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 96, 128, 64, f(1.0), 3, None, None) == -2
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

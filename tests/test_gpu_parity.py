@@ -30,31 +30,33 @@ def _lib(cuda_device):
     assert api.device_status() == 0
 
 
-def gpu_run(Q, K, V, block, beta):
+def gpu_run(Q, K, V, block, beta, diagonal=False):
     out = torch.full_like(Q, float("nan"))
-    api.forward(Q, K, V, beta, block, out=out)
-    counts, sel = api.stats(Q, K, beta, block, with_mask=True)
+    api.forward_ex(Q, K, V, beta, block, out=out, diagonal_sigma=diagonal)
+    counts, sel = api.stats(Q, K, beta, block, with_mask=True, diagonal_sigma=diagonal)
     torch.cuda.synchronize()
     return out, counts.cpu().numpy(), sel.cpu().numpy()
 
 
-def check_case(Q, K, V, block, beta, sample_k=None, extra_blocks=(), seed=0, heads=None):
+def check_case(Q, K, V, block, beta, sample_k=None, extra_blocks=(), seed=0, heads=None, diagonal=False):
     """Runs the GPU forward + stats and checks them against the oracle."""
     b_, H, L, d = Q.shape
-    out, counts, sel = gpu_run(Q, K, V, block, beta)
+    bq, bk = P.pair(block)
+    moments = "diagonal" if diagonal else "eq5"
+    out, counts, sel = gpu_run(Q, K, V, block, beta, diagonal)
     rng = np.random.default_rng(seed)
     stats = []
     gpu_rows, ref_rows = [], []
     for b in range(b_):
         for h in range(H) if heads is None else heads:
-            r = O.route_head(P.head_np(Q, b, h), P.head_np(K, b, h), block, block, beta)
+            r = O.route_head(P.head_np(Q, b, h), P.head_np(K, b, h), bq, bk, beta, moments)
             stats.append(P.compare_selection(r, sel[b, h], counts[b, h]))
             N = r["qgeom"].n
             if sample_k is None:
                 blocks = list(range(N))
             else:
                 blocks = P.sample_blocks(N, counts[b, h], sample_k, rng, extra_blocks)
-            ref = P.oracle_rows(Q, K, V, b, h, block, beta, sel[b, h], blocks)
+            ref = P.oracle_rows(Q, K, V, b, h, block, beta, sel[b, h], blocks, moments)
             rows = P.rows_of(blocks, block, L)
             ref_rows.append(ref[rows])
             gpu_rows.append(out[b, h].double().cpu().numpy()[rows])
@@ -81,10 +83,11 @@ def test_tiny_fp32_workload(beta):
 
 
 @pytest.mark.parametrize("L", [1, 5, 127, 128, 129, 300])
+@pytest.mark.parametrize("block", [128, (128, 64)])
 @pytest.mark.parametrize("beta", [-INF, 1.04, INF])
-def test_short_and_ragged_lengths(L, beta):
+def test_short_and_ragged_lengths(L, beta, block):
     Q, K, V = I.make_iid(1, 3, L, 128, seed=L, dtype=torch.bfloat16, device="cuda")
-    check_case(Q, K, V, 128, beta)
+    check_case(Q, K, V, block, beta)
 
 
 @pytest.mark.parametrize("d,block,dtype", [(128, 128, torch.float32), (64, 64, torch.bfloat16),
@@ -94,6 +97,48 @@ def test_other_shapes(d, block, dtype):
     Q, K, V = I.make_qkv((3, 12, 20), heads=2, d=d, seed=11, dtype=dtype, device="cuda")  # L = 720
     for beta in (-INF, 0.7, INF):
         check_case(Q, K, V, block, beta)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("bq,bk", [(128, 64), (64, 128)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_query_and_key_blocks_of_different_sizes(bq, bk, d, dtype):
+    # L = 1000: ragged query and key tails of different lengths (104/40 tokens)
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=d, seed=12, dtype=dtype, device="cuda")
+    for beta in (-INF, 0.5, 1.04, INF):
+        err, _ = check_case(Q, K, V, (bq, bk), beta)
+        if dtype == torch.float32:
+            assert err["rel_l2"] <= 1e-4
+
+
+@pytest.mark.parametrize("block", [128, 64, (128, 64)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_diagonal_sigma(block, dtype):
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=13, dtype=dtype, device="cuda")
+    for beta in (-1.0, 0.5, 1.04, 2.0):
+        check_case(Q, K, V, block, beta, diagonal=True)
+
+
+def test_diagonal_sigma_video_workload():
+    """Wan2.1 480p shape: every selection row against the oracle's diagonal
+    routing; sampled output rows; the selected fraction moves with the
+    estimator but stays in the same range."""
+    wl = I.WORKLOADS["wan-480p"]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    out, counts, sel = gpu_run(Q, K, V, wl.block, 1.04, diagonal=True)
+    rng = np.random.default_rng(4)
+    gpu_rows, ref_rows = [], []
+    for h in range(wl.heads):
+        r = O.route_head(P.head_np(Q, 0, h), P.head_np(K, 0, h), wl.block, wl.block, 1.04, "diagonal")
+        P.compare_selection(r, sel[0, h], counts[0, h])
+        if h in (0, wl.heads - 1):
+            blocks = P.sample_blocks(wl.n_blocks, counts[0, h], 8, rng)
+            ref = P.oracle_rows(Q, K, V, 0, h, wl.block, 1.04, sel[0, h], blocks, "diagonal")
+            rows = P.rows_of(blocks, wl.block, wl.L)
+            ref_rows.append(ref[rows])
+            gpu_rows.append(out[0, h].double().cpu().numpy()[rows])
+    P.check_close(np.concatenate(gpu_rows), np.concatenate(ref_rows), Q.dtype, "wan-480p diagonal")
+    assert 0.02 < sel.mean() < 0.40
 
 
 @pytest.mark.parametrize("beta", [-INF, 0.0, 1.04, INF])
@@ -137,14 +182,18 @@ def test_image_dit(beta):
     check_case(Q, K, V, wl.block, beta, sample_k=3, heads=range(wl.heads), seed=1)
 
 
-@pytest.mark.parametrize("name,beta", [("wan-480p", 1.04),
-                                       ("wan-720p", -INF), ("wan-720p", 0.5), ("wan-720p", 1.04),
-                                       ("wan-720p", 1.5), ("wan-720p", 2.0),
-                                       ("hunyuan-720p", 1.04), ("hunyuan-720p", 1.5)])
-def test_video_workloads(name, beta):
+@pytest.mark.parametrize("name,beta,bk", [("wan-480p", 1.04, 128),
+                                          ("wan-720p", -INF, 128), ("wan-720p", 0.5, 128), ("wan-720p", 1.04, 128),
+                                          ("wan-720p", 1.5, 128), ("wan-720p", 2.0, 128),
+                                          ("hunyuan-720p", 1.04, 128), ("hunyuan-720p", 1.5, 128),
+                                          # key blocks of 64 tokens, two per tensor-core tile
+                                          ("wan-480p", 1.04, 64), ("wan-720p", 1.04, 64), ("wan-720p", -INF, 64),
+                                          ("hunyuan-720p", 1.04, 64)])
+def test_video_workloads(name, beta, bk):
     wl = I.WORKLOADS[name]
+    block = (wl.block, bk)
     Q, K, V = I.make_workload(wl, device="cuda")
-    out, counts, sel = gpu_run(Q, K, V, wl.block, beta)
+    out, counts, sel = gpu_run(Q, K, V, block, beta)
     assert not torch.isnan(out).any()
     rng = np.random.default_rng(2)
     N = wl.n_blocks
@@ -156,12 +205,12 @@ def test_video_workloads(name, beta):
     gpu_rows, ref_rows = [], []
     for h in range(wl.heads):
         Qh, Kh = P.head_np(Q, 0, h), P.head_np(K, 0, h)
-        r = O.route_head(Qh, Kh, wl.block, wl.block, beta)
+        r = O.route_head(Qh, Kh, wl.block, bk, beta)
         P.compare_selection(r, sel[0, h], counts[0, h])
         if h in sample_heads:
             k = 12 if beta != -INF else 4
             blocks = P.sample_blocks(N, counts[0, h], k, rng, text_blocks)
-            ref = P.oracle_rows(Q, K, V, 0, h, wl.block, beta, sel[0, h], blocks)
+            ref = P.oracle_rows(Q, K, V, 0, h, block, beta, sel[0, h], blocks)
             rows = P.rows_of(blocks, wl.block, wl.L)
             ref_rows.append(ref[rows])
             gpu_rows.append(out[0, h].double().cpu().numpy()[rows])
@@ -174,6 +223,7 @@ def test_video_workloads(name, beta):
 # ------------------------------------------------------------------ keep-or-drop (correction off)
 
 def check_keep_or_drop(Q, K, V, block, beta):
+    bq, bk = P.pair(block)
     out = torch.full_like(Q, float("nan"))
     api.forward_ex(Q, K, V, beta, block, out=out, keep_or_drop=True)
     counts, sel = api.stats(Q, K, beta, block, with_mask=True)
@@ -183,9 +233,9 @@ def check_keep_or_drop(Q, K, V, block, beta):
     gpu_rows, ref_rows = [], []
     for b in range(Q.shape[0]):
         for h in range(Q.shape[1]):
-            r = O.route_head(P.head_np(Q, b, h), P.head_np(K, b, h), block, block, beta)
+            r = O.route_head(P.head_np(Q, b, h), P.head_np(K, b, h), bq, bk, beta)
             P.compare_selection(r, sel[b, h], counts[b, h])
-            ref, _ = O.forward_head(P.head_np(Q, b, h), P.head_np(K, b, h), P.head_np(V, b, h), block, block,
+            ref, _ = O.forward_head(P.head_np(Q, b, h), P.head_np(K, b, h), P.head_np(V, b, h), bq, bk,
                                     beta, sel=sel[b, h], correction=False)
             ref_rows.append(ref)
             gpu_rows.append(out[b, h].double().cpu().numpy())
@@ -193,10 +243,11 @@ def check_keep_or_drop(Q, K, V, block, beta):
     return P.check_close(np.concatenate(gpu_rows), np.concatenate(ref_rows), Q.dtype, f"keep-or-drop beta={beta}")
 
 
+@pytest.mark.parametrize("block", [128, (128, 64)])
 @pytest.mark.parametrize("beta", [-INF, 0.5, 1.04, 2.0, INF])
-def test_keep_or_drop_bf16(beta):
+def test_keep_or_drop_bf16(beta, block):
     Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=8, device="cuda")  # L = 1000, ragged tail
-    check_keep_or_drop(Q, K, V, 128, beta)
+    check_keep_or_drop(Q, K, V, block, beta)
 
 
 @pytest.mark.parametrize("beta", [0.5, 1.04, INF])

@@ -21,9 +21,10 @@ STATUS = {0: "SOL_OK", -1: "SOL_ERR_INVALID_ARG", -2: "SOL_ERR_UNSUPPORTED", -3:
           -4: "SOL_ERR_NO_MEMORY", -5: "SOL_ERR_DEVICE_TIMEOUT"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 FLAG_KEEP_OR_DROP = 1  # correction off: unselected blocks contribute nothing
+FLAG_DIAGONAL_SIGMA = 2  # sigma_i from the diagonal moment estimator
 
 EXPORTS = ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
-           "sol_attn_device_status", "sol_attn_status_string", "sol_attn_version")
+           "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_status_string", "sol_attn_version")
 
 
 class SolAttnError(RuntimeError):
@@ -46,12 +47,15 @@ def lib() -> ctypes.CDLL:
                                           vp, vp]
         L.sol_attn_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.sol_attn_stats.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
+        L.sol_attn_stats_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, ctypes.c_uint,
+                                        vp]
         L.sol_attn_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         L.sol_attn_status_string.argtypes = [i32]
         L.sol_attn_status_string.restype = ctypes.c_char_p
         L.sol_attn_version.argtypes = []
         for name in ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
-                     "sol_attn_device_status", "sol_attn_version", "sol_attn_forward_noalloc"):
+                     "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_version",
+                     "sol_attn_forward_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -86,28 +90,40 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
-def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, block: int = 128,
+def blocks(block) -> tuple[int, int]:
+    """(Bq, Bk) from a block size or a (query, key) pair."""
+    if isinstance(block, (tuple, list)):
+        bq, bk = block
+        return int(bq), int(bk)
+    return int(block), int(block)
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, block=128,
             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Sol-Attn forward of [batch, heads, L, d] bf16 or fp32 tensors."""
+    """Sol-Attn forward of [batch, heads, L, d] bf16 or fp32 tensors; block is
+    one size for query and key blocks or a (Bq, Bk) pair."""
     b, h, L, d = _shape(q, k, v)
+    bq, bk = blocks(block)
     if out is None:
         out = torch.empty_like(q)
     fn = lib().sol_attn_forward if q.dtype == torch.bfloat16 else lib().sol_attn_forward_f32
     _dtype_code(q)
-    rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b, h, L, d, block, block,
+    rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b, h, L, d, bq, bk,
             float(beta), _stream_handle(stream))
     _check("sol_attn_forward", rc)
     return out
 
 
-def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, stream=None,
-               keep_or_drop: bool = False) -> torch.Tensor:
+def forward_ex(q, k, v, beta: float, block=128, out=None, events=None, stream=None,
+               keep_or_drop: bool = False, diagonal_sigma: bool = False) -> torch.Tensor:
     """forward() that also records up to four torch.cuda.Event objects: before
     pooling, after pooling, after routing, after the attention kernel.  The
     events must exist already (torch creates them on their first record()).
     keep_or_drop=True switches the correction off (unselected blocks
-    contribute nothing; rows with no selected block give 0)."""
+    contribute nothing; rows with no selected block give 0); diagonal_sigma=True
+    takes sigma_i from the diagonal moment estimator."""
     b, h, L, d = _shape(q, k, v)
+    bq, bk = blocks(block)
     if out is None:
         out = torch.empty_like(q)
     ev = None
@@ -119,29 +135,32 @@ def forward_ex(q, k, v, beta: float, block: int = 128, out=None, events=None, st
                 raise ValueError("event not created yet: record it once before passing it")
         ev = ctypes.cast(arr, ctypes.c_void_p)
     rc = lib().sol_attn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
-                                   b, h, L, d, block, block, float(beta),
-                                   FLAG_KEEP_OR_DROP if keep_or_drop else 0, ev, _stream_handle(stream))
+                                   b, h, L, d, bq, bk, float(beta),
+                                   (FLAG_KEEP_OR_DROP if keep_or_drop else 0)
+                                   | (FLAG_DIAGONAL_SIGMA if diagonal_sigma else 0), ev, _stream_handle(stream))
     _check("sol_attn_forward_ex", rc)
     return out
 
 
-def stats(q: torch.Tensor, k: torch.Tensor, beta: float, block: int = 128, with_mask: bool = False,
-          stream=None):
+def stats(q: torch.Tensor, k: torch.Tensor, beta: float, block=128, with_mask: bool = False,
+          stream=None, diagonal_sigma: bool = False):
     """Selected-block counts [batch, heads, Nq] (int32) and, if asked, the
     selection as a bool tensor [batch, heads, Nq, Nk] unpacked from the
     library's 1-bit mask."""
     b, h, L, d = _shape(q, k)
-    N = -(-L // block)
-    W = -(-N // 32)
-    counts = torch.empty(b, h, N, dtype=torch.int32, device=q.device)
-    mask = torch.empty(b, h, N, W, dtype=torch.int32, device=q.device) if with_mask else None
-    rc = lib().sol_attn_stats(q.data_ptr(), k.data_ptr(), counts.data_ptr(),
-                              mask.data_ptr() if mask is not None else None, b, h, L, d, block, block,
-                              float(beta), _dtype_code(q), _stream_handle(stream))
-    _check("sol_attn_stats", rc)
+    bq, bk = blocks(block)
+    Nq, Nk = -(-L // bq), -(-L // bk)
+    W = -(-Nk // 32)
+    counts = torch.empty(b, h, Nq, dtype=torch.int32, device=q.device)
+    mask = torch.empty(b, h, Nq, W, dtype=torch.int32, device=q.device) if with_mask else None
+    rc = lib().sol_attn_stats_ex(q.data_ptr(), k.data_ptr(), counts.data_ptr(),
+                                 mask.data_ptr() if mask is not None else None, b, h, L, d, bq, bk,
+                                 float(beta), _dtype_code(q), FLAG_DIAGONAL_SIGMA if diagonal_sigma else 0,
+                                 _stream_handle(stream))
+    _check("sol_attn_stats_ex", rc)
     if mask is None:
         return counts
-    return counts, unpack_mask(mask, N)
+    return counts, unpack_mask(mask, Nk)
 
 
 def unpack_mask(words: torch.Tensor, N: int) -> torch.Tensor:

@@ -29,23 +29,25 @@ int check_args(const void* q, const void* k, const void* v_or_dummy, const void*
   if (batch < 1 || heads < 1 || L < 1 || d < 1 || Bq < 1 || Bk < 1) return SOL_ERR_INVALID_ARG;
   if (std::isnan(beta)) return SOL_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SOL_ERR_UNSUPPORTED;
-  if (Bq != Bk) return SOL_ERR_UNSUPPORTED;
-  if (Bq != 64 && Bq != 128) return SOL_ERR_UNSUPPORTED;
+  if ((Bq != 64 && Bq != 128) || (Bk != 64 && Bk != 128)) return SOL_ERR_UNSUPPORTED;
   const int64_t bH = (int64_t)batch * heads;
   if (bH > (1 << 24) || bH * (int64_t)L * d >= (int64_t(1) << 40)) return SOL_ERR_UNSUPPORTED;
-  const int B = Bq;
-  const int N = (L + B - 1) / B;
-  if (N > sol::kRouteMaxN) return SOL_ERR_UNSUPPORTED;
-  if (bH * N >= (int64_t(1) << 31)) return SOL_ERR_UNSUPPORTED;
+  const int Nq = (L + Bq - 1) / Bq;
+  const int Nk = (L + Bk - 1) / Bk;
+  if (Nk > sol::kRouteMaxN) return SOL_ERR_UNSUPPORTED;
+  if (bH * Nq >= (int64_t(1) << 31) || bH * Nk >= (int64_t(1) << 31)) return SOL_ERR_UNSUPPORTED;
   g->bH = (int)bH;
   g->L = L;
   g->d = d;
-  g->B = B;
-  g->N = N;
-  g->W = (N + 31) / 32;
-  g->nchunk = (N + B - 1) / B;
-  g->n_last = L - (N - 1) * B;
-  g->nitems = (int)(bH * N);
+  g->Bq = Bq;
+  g->Bk = Bk;
+  g->Nq = Nq;
+  g->Nk = Nk;
+  g->W = (Nk + 31) / 32;
+  g->nchunk = (Nk + sol::kChunk - 1) / sol::kChunk;
+  g->nq_last = L - (Nq - 1) * Bq;
+  g->nk_last = L - (Nk - 1) * Bk;
+  g->nitems = (int)(bH * Nq);
   return SOL_OK;
 }
 
@@ -53,17 +55,19 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Carves the scratch out of one allocation; returns its size when base is null.
 size_t carve(const Geometry& g, size_t op_elem, char* base, Scratch* s) {
-  const size_t pooled = (size_t)g.bH * g.N * g.d;
+  const size_t qpooled = (size_t)g.bH * g.Nq * g.d;
+  const size_t kpooled = (size_t)g.bH * g.Nk * g.d;
   size_t off = 0;
   auto take = [&](size_t bytes) -> char* {
     char* p = base ? base + off : nullptr;
     off += align256(bytes);
     return p;
   };
-  s->qbar = reinterpret_cast<float*>(take(pooled * sizeof(float)));
-  s->kbar = reinterpret_cast<float*>(take(pooled * sizeof(float)));
-  s->kbar_op = take(pooled * op_elem);
-  s->vbar_op = take(pooled * op_elem);
+  s->qbar = reinterpret_cast<float*>(take(qpooled * sizeof(float)));
+  s->kbar = reinterpret_cast<float*>(take(kpooled * sizeof(float)));
+  s->kbar_op = take(kpooled * op_elem);
+  s->vbar_op = take(kpooled * op_elem);
+  s->kvar = reinterpret_cast<float*>(take((size_t)g.bH * g.d * sizeof(float)));
   s->mask = reinterpret_cast<uint32_t*>(take((size_t)g.nitems * g.W * sizeof(uint32_t)));
   s->counts = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
   s->tiles = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
@@ -104,6 +108,14 @@ cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
   return cudaMallocFromPoolAsync(p, bytes, pool, st);
 }
 
+// The tensor-core kernel is built for bf16 with d = 128, query blocks of 128
+// tokens and key blocks of 128 or 64 (two 64-token blocks share one tile).
+bool uses_tensor_cores(int dtype, const Geometry& g) {
+  return dtype == SOL_DTYPE_BF16 && g.d == 128 && g.Bq == 128 && (g.Bk == 128 || g.Bk == 64);
+}
+
+int pair_tiles(bool use_tc, const Geometry& g) { return use_tc && g.Bk == 64 ? 1 : 0; }
+
 int beta_mode_of(float beta) { return std::isinf(beta) ? (beta < 0 ? -1 : 1) : 0; }
 
 uint64_t wait_limit_ns() {
@@ -124,12 +136,13 @@ int record(void* const* events, int i, cudaStream_t st) {
 int forward_impl(const void* q, const void* k, const void* v, void* out, int dtype, int batch, int heads, int L,
                  int d, int Bq, int Bk, float beta, unsigned flags, void* const* events, cudaStream_t st) {
   if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
-  if (flags & ~SOL_FLAG_KEEP_OR_DROP) return SOL_ERR_INVALID_ARG;
+  if (flags & ~(SOL_FLAG_KEEP_OR_DROP | SOL_FLAG_DIAGONAL_SIGMA)) return SOL_ERR_INVALID_ARG;
   const int correction = (flags & SOL_FLAG_KEEP_OR_DROP) ? 0 : 1;
+  const int sigma_mode = (flags & SOL_FLAG_DIAGONAL_SIGMA) ? sol::kSigmaDiagonal : sol::kSigmaEq5;
   Geometry g;
   int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
   if (rc != SOL_OK) return rc;
-  const bool use_tc = dtype == SOL_DTYPE_BF16 && g.d == 128 && g.B == 128;
+  const bool use_tc = uses_tensor_cores(dtype, g);
   const int op_dtype = use_tc ? 0 : 1;  // operand type of K-bar / V-bar: bf16 for tensor cores
   Scratch s;
   const size_t bytes = carve(g, use_tc ? 2 : 4, nullptr, &s);
@@ -145,7 +158,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   e = sol::launch_pool(in_dtype, op_dtype, q, k, v, g, s, st);
   if (e != cudaSuccess) goto done;
   if ((rc = record(events, 1, st)) != SOL_OK) goto done;
-  e = sol::launch_route(g, s, beta, beta_mode_of(beta), correction, st);
+  e = sol::launch_route(g, s, beta, beta_mode_of(beta), correction, sigma_mode, pair_tiles(use_tc, g), st);
   if (e != cudaSuccess) goto done;
   e = sol::launch_order(g, s, st);
   if (e != cudaSuccess) goto done;
@@ -188,10 +201,12 @@ int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, 
                       static_cast<cudaStream_t>(stream));
 }
 
-int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int batch, int heads,
-                   int L, int d, int Bq, int Bk, float beta, int dtype, void* stream) {
+int sol_attn_stats_ex(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int batch, int heads,
+                      int L, int d, int Bq, int Bk, float beta, int dtype, unsigned int flags, void* stream) {
   if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
   if (!counts) return SOL_ERR_INVALID_ARG;
+  if (flags & ~SOL_FLAG_DIAGONAL_SIGMA) return SOL_ERR_INVALID_ARG;
+  const int sigma_mode = (flags & SOL_FLAG_DIAGONAL_SIGMA) ? sol::kSigmaDiagonal : sol::kSigmaEq5;
   Geometry g;
   int rc = check_args(q, k, q, q, batch, heads, L, d, Bq, Bk, beta, &g);
   if (rc != SOL_OK) return rc;
@@ -208,9 +223,14 @@ int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask
   if (mask_or_null) s.mask = mask_or_null;
   s.kbar_op = nullptr;  // routing needs the fp32 pooled vectors only
   cudaError_t e = sol::launch_pool(dtype == SOL_DTYPE_BF16 ? 0 : 1, 1, q, k, nullptr, g, s, st);
-  if (e == cudaSuccess) e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, st);
+  if (e == cudaSuccess) e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, sigma_mode, 0, st);
   cudaFreeAsync(base, st);
   return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+}
+
+int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int batch, int heads,
+                   int L, int d, int Bq, int Bk, float beta, int dtype, void* stream) {
+  return sol_attn_stats_ex(q, k, counts, mask_or_null, batch, heads, L, d, Bq, Bk, beta, dtype, 0u, stream);
 }
 
 int sol_attn_device_status(void* stream, int32_t* detail) {
@@ -232,7 +252,7 @@ const char* sol_attn_status_string(int status) {
   }
 }
 
-int sol_attn_version(void) { return 101; }
+int sol_attn_version(void) { return 102; }
 
 }  // extern "C"
 
@@ -285,7 +305,7 @@ extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void
   Geometry g;
   int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
   if (rc != SOL_OK) return rc;
-  const bool use_tc = g.d == 128 && g.B == 128;
+  const bool use_tc = uses_tensor_cores(SOL_DTYPE_BF16, g);
   const int op_dtype = use_tc ? 0 : 1;
   Scratch s;
   const size_t bytes = carve(g, use_tc ? 2 : 4, nullptr, &s);
@@ -297,7 +317,8 @@ extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void
   // Everything the kernels read is rewritten by this call except the work
   // counter, which must start at zero.
   cudaError_t e = sol::launch_pool(0, op_dtype, q, k, v, g, s, st);
-  if (e == cudaSuccess) e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, st);
+  if (e == cudaSuccess)
+    e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, sol::kSigmaEq5, pair_tiles(use_tc, g), st);
   if (e == cudaSuccess) e = sol::launch_order(g, s, st);
   if (use_tc) {
     if (e == cudaSuccess) e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);

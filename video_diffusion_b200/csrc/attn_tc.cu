@@ -1,5 +1,6 @@
 // attn_tc.cu -- the Sol-Attn attention loop on the 5th-generation tensor cores
-// (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, d = 128, B = 128.
+// (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, d = 128, query
+// blocks of 128 tokens, key blocks of 128 or 64 tokens.
 //
 // The MMA warp's barrier operations, not the tensor pipe, set the pace of
 // the key loop (each wait or commit costs a few hundred cycles while the
@@ -16,7 +17,9 @@
 //     softmax column; selected and out-of-range columns are masked out;
 //   * then each selected key block j in increasing order: S = Q_i K_j^T, masked
 //     past the block's n_j tokens, and O += P V_j (Eqs. 9, 10 "Exact" terms).
-//     Only selected K/V tiles are ever loaded.
+//     Only selected K/V tiles are ever loaded.  With 64-token key blocks one
+//     128-column tile holds two selected blocks, one per softmax column half
+//     (an odd count leaves the last tile's second half masked out).
 //
 // Persistent CTAs, one per SM, 320 threads:
 //   warp 0      TMA producer: fetches work items, loads the Q tile and each
@@ -74,10 +77,11 @@ __host__ __device__ constexpr bool poly_pair(int pair) {
 }
 
 struct Params {
-  int bH, L, N, W, nchunk, nitems, n_last;
+  int bH, L, Nq, Nk, W, nchunk, nitems, nk_last;
+  int pair;             // 1: key blocks of 64 tokens, two per exact tile; 0: blocks of 128
   float scale_log2;     // log2(e) / sqrt(d)
-  float bias_full;      // log2(B)
-  float bias_last;      // log2(n_last)
+  float bias_full;      // log2(Bk)
+  float bias_last;      // log2(nk_last)
   const uint32_t* mask;
   const int32_t* tiles;
   const int32_t* order;
@@ -108,23 +112,35 @@ static_assert(sizeof(Bars) <= BAR_AREA, "barrier area");
 static_assert(QST == 1, "one Q buffer");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
-// unselected block, then the selected blocks in increasing order.
+// unselected block, then the selected blocks in increasing order (one per
+// tile, or two with 64-token key blocks).
 struct TileIter {
   const uint32_t* m;
-  int W, N, nchunk;
+  int W, N, nchunk, pair;
   int chunk;     // next chunk to test
   int word;      // current mask word in the exact phase
   uint32_t bits; // remaining set bits of that word
-  __device__ void init(const uint32_t* mrow, int W_, int N_, int nchunk_) {
-    m = mrow; W = W_; N = N_; nchunk = nchunk_;
+  __device__ void init(const uint32_t* mrow, int W_, int N_, int nchunk_, int pair_) {
+    m = mrow; W = W_; N = N_; nchunk = nchunk_; pair = pair_;
     chunk = 0; word = -1; bits = 0;
+  }
+  __device__ __forceinline__ int next_selected() {
+    while (bits == 0) {
+      if (++word >= W) return -1;
+      bits = m[word];
+    }
+    const int b = __ffs(bits) - 1;
+    bits &= bits - 1;
+    return word * 32 + b;
   }
   __device__ __forceinline__ uint32_t valid_bits(int w) const {
     const int nb = N - w * 32;
     return nb >= 32 ? 0xffffffffu : (nb <= 0 ? 0u : ((1u << nb) - 1u));
   }
-  // kind 0: pooled chunk idx; kind 1: exact key block idx.  false when done.
-  __device__ bool next(int& kind, int& idx) {
+  // kind 0: pooled chunk idx; kind 1: exact key block idx (and, in pair mode,
+  // idx2 = the second block of the tile or -1).  false when done.
+  __device__ bool next(int& kind, int& idx, int& idx2) {
+    idx2 = -1;
     while (chunk < nchunk) {
       const int c = chunk++;
       uint32_t un = 0;
@@ -135,14 +151,10 @@ struct TileIter {
       }
       if (un) { kind = 0; idx = c; return true; }
     }
-    while (bits == 0) {
-      if (++word >= W) return false;
-      bits = m[word];
-    }
-    const int b = __ffs(bits) - 1;
-    bits &= bits - 1;
+    idx = next_selected();
+    if (idx < 0) return false;
+    if (pair) idx2 = next_selected();
     kind = 1;
-    idx = word * 32 + b;
     return true;
   }
 };
@@ -256,7 +268,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&bars.item_full[slot]);
       }
       if (item < 0) break;
-      const int bh = item / p.N, qi = item % p.N;
+      const int bh = item / p.Nq, qi = item % p.Nq;
       const int T = p.tiles[item];
       if (T == 0) continue;
       // Q tile into buffer q_uses % QST, once the item that used it last has
@@ -272,10 +284,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       ++q_uses;
       TileIter ti;
-      ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.chunks);
+      ti.init(p.mask + (size_t)item * p.W, p.W, p.Nk, p.chunks, p.pair);
       for (int n = 0; n < T; ++n) {
-        int kind = 0, tidx = 0;
-        ti.next(kind, tidx);
+        int kind = 0, tidx = 0, tidx2 = -1;
+        ti.next(kind, tidx, tidx2);
         const uint32_t gk = g + n;
         const int ks = gk % KVST;
         const int ku = gk / KVST;
@@ -285,12 +297,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint8_t* dk = smem + OFF_KV + (2 * ks) * TILE_BYTES;
           uint8_t* dv = dk + TILE_BYTES;
           mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
-          const CUtensorMap* mk = kind ? &tmK : &tmKb;
-          const CUtensorMap* mv = kind ? &tmV : &tmVb;
-          tma_load_3d(dk, mk, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
-          tma_load_3d(dk + HALF_BYTES, mk, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
-          tma_load_3d(dv, mv, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
-          tma_load_3d(dv + HALF_BYTES, mv, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
+          if (kind == 1 && p.pair) {
+            // rows [0, 64) <- key block tidx, rows [64, 128) <- key block tidx2;
+            // a tile with one block repeats it in the second half (masked out)
+            const int j2 = tidx2 >= 0 ? tidx2 : tidx;
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+              tma_load_3d(dk + hd * HALF_BYTES, &tmK, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+              tma_load_3d(dk + hd * HALF_BYTES + 64 * 128, &tmK, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+              tma_load_3d(dv + hd * HALF_BYTES, &tmV, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+              tma_load_3d(dv + hd * HALF_BYTES + 64 * 128, &tmV, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+            }
+          } else {
+            const CUtensorMap* mk = kind ? &tmK : &tmKb;
+            const CUtensorMap* mv = kind ? &tmV : &tmVb;
+            tma_load_3d(dk, mk, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
+            tma_load_3d(dk + HALF_BYTES, mk, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
+            tma_load_3d(dv, mv, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
+            tma_load_3d(dv + HALF_BYTES, mv, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
+          }
         }
         gk_last = (int)gk;
       }
@@ -414,7 +439,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (item < 0) break;
-      const int bh = item / p.N, qi = item % p.N;
+      const int bh = item / p.Nq, qi = item % p.Nq;
       const int T = p.tiles[item];
       const int n_rows = min(BM, p.L - qi * BM);
       __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD + col0;
@@ -424,11 +449,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         continue;
       }
       TileIter ti;
-      ti.init(p.mask + (size_t)item * p.W, p.W, p.N, p.chunks);
+      ti.init(p.mask + (size_t)item * p.W, p.W, p.Nk, p.chunks, p.pair);
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < T; ++n) {
-        int kind = 0, tidx = 0;
-        ti.next(kind, tidx);
+        int kind = 0, tidx = 0, tidx2 = -1;
+        ti.next(kind, tidx, tidx2);
         const uint32_t gs = g + n;
         const int pb = gs & 1;
         if (!(ok = wait_warp(&bars.s_full, gs & 1, bars, lim, 21))) break;
@@ -449,9 +474,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_free);
 
+        // valid key columns of this half of an exact tile: all 64 except in
+        // the last (partial) key block and in a pair tile's empty second half
+        int nvalid = 64;
+        if (kind == 1) {
+          if (p.pair) {
+            const int jh = half ? tidx2 : tidx;
+            nvalid = jh < 0 ? 0 : (jh == p.Nk - 1 ? p.nk_last : 64);
+          } else {
+            const int nblk = tidx == p.Nk - 1 ? p.nk_last : BN;
+            nvalid = min(max(nblk - col0, 0), 64);
+          }
+        }
         // full exact tile: x stays the raw score (scale folded into exp2 below);
         // otherwise x becomes the log2-domain logit with bias and mask applied
-        const bool full = kind == 1 && (tidx != p.N - 1 || p.n_last == BN);
+        const bool full = kind == 1 && nvalid == 64;
         float lmax;
         if (full) {
           lmax = tree_max64(x) * sl2;  // scaling by sl2 > 0 commutes with max
@@ -460,10 +497,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float bias = 0.f;
           int sc = -1;
           float sc_delta = 0.f;
-          if (kind == 1) {  // partial last key block: columns >= n_last are padding
+          if (kind == 1) {  // columns past the valid ones are padding
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-              const int nb = p.n_last - col0 - q * 32;
+              const int nb = nvalid - q * 32;
               vm[q] = nb >= 32 ? ~0u : (nb <= 0 ? 0u : ((1u << nb) - 1u));
             }
           } else {  // pooled chunk: unselected, in-range blocks only
@@ -473,8 +510,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const int w = tidx * 4 + half * 2 + q;
               vm[q] = (w < p.W) ? ((~p.mask[(size_t)item * p.W + w]) & ti.valid_bits(w)) : 0u;
             }
-            const int jl = p.N - 1 - tidx * BN - col0;
-            if (jl >= 0 && jl < 64 && p.n_last != BN) {
+            const int jl = p.Nk - 1 - tidx * BN - col0;
+            if (jl >= 0 && jl < 64 && p.bias_last != p.bias_full) {
               sc = jl;
               sc_delta = p.bias_last - p.bias_full;
             }
@@ -621,14 +658,14 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [planes, rows, 128] bf16 tensor, boxes of 64 columns x 128 rows, 128-byte
-// swizzle; rows past `rows` read as zero.
-bool make_map(CUtensorMap* m, const void* base, int rows, int planes) {
+// [planes, rows, 128] bf16 tensor, boxes of 64 columns x box_rows rows,
+// 128-byte swizzle; rows past `rows` read as zero.
+bool make_map(CUtensorMap* m, const void* base, int rows, int planes, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)rows, (cuuint64_t)planes};
   cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)rows * HD * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -640,14 +677,19 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int planes) {
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
                            const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction) {
   CUtensorMap mQ, mK, mV, mKb, mVb;
-  if (!make_map(&mQ, q, g.L, g.bH) || !make_map(&mK, k, g.L, g.bH) || !make_map(&mV, v, g.L, g.bH) ||
-      !make_map(&mKb, s.kbar_op, g.N, g.bH) || !make_map(&mVb, s.vbar_op, g.N, g.bH))
+  // built for d == 128, query blocks of 128 tokens, key blocks of 128 or 64
+  if (g.Bq != BM || (g.Bk != BN && g.Bk != BN / 2) || g.d != HD) return cudaErrorInvalidValue;
+  if (!make_map(&mQ, q, g.L, g.bH, BM) || !make_map(&mK, k, g.L, g.bH, g.Bk) ||
+      !make_map(&mV, v, g.L, g.bH, g.Bk) || !make_map(&mKb, s.kbar_op, g.Nk, g.bH, BN) ||
+      !make_map(&mVb, s.vbar_op, g.Nk, g.bH, BN))
     return cudaErrorInvalidValue;
   Params p;
-  p.bH = g.bH; p.L = g.L; p.N = g.N; p.W = g.W; p.nchunk = g.nchunk; p.nitems = g.nitems; p.n_last = g.n_last;
+  p.bH = g.bH; p.L = g.L; p.Nq = g.Nq; p.Nk = g.Nk; p.W = g.W; p.nchunk = g.nchunk; p.nitems = g.nitems;
+  p.nk_last = g.nk_last;
+  p.pair = g.Bk == BN / 2 ? 1 : 0;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
-  p.bias_full = (float)std::log2((double)g.B);
-  p.bias_last = (float)std::log2((double)g.n_last);
+  p.bias_full = (float)std::log2((double)g.Bk);
+  p.bias_last = (float)std::log2((double)g.nk_last);
   p.mask = s.mask; p.tiles = s.tiles; p.order = s.order; p.work_counter = s.work_counter;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.wait_limit_ns = wait_limit_ns;

@@ -7,41 +7,55 @@
 
 namespace sol {
 
-// Geometry of one call.  Bq == Bk == B; blocks are contiguous runs of B
-// tokens in sequence order and the last one holds n_last = L - (N-1) B tokens.
+// Geometry of one call.  Query and key blocks are contiguous runs of Bq and
+// Bk tokens in sequence order; the last query block holds nq_last tokens and
+// the last key block nk_last.
 struct Geometry {
-  int bH;      // batch * heads
-  int L;       // tokens
-  int d;       // head dimension
-  int B;       // block size (query and key)
-  int N;       // blocks per head, ceil(L / B)
-  int W;       // 32-bit words per selection-mask row, ceil(N / 32)
-  int nchunk;  // pooled-key chunks of B pooled keys, ceil(N / B)
-  int n_last;  // tokens in the last block
-  int nitems;  // bH * N work items (one per query block)
+  int bH;       // batch * heads
+  int L;        // tokens
+  int d;        // head dimension
+  int Bq, Bk;   // query / key block size
+  int Nq, Nk;   // blocks per head: ceil(L / Bq), ceil(L / Bk)
+  int W;        // 32-bit words per selection-mask row, ceil(Nk / 32)
+  int nchunk;   // chunks of kChunk pooled keys, ceil(Nk / kChunk)
+  int nq_last;  // tokens in the last query block
+  int nk_last;  // tokens in the last key block
+  int nitems;   // bH * Nq work items (one per query block)
 };
+
+// Pooled keys per chunk of the approximate path: one 128-column score tile of
+// the tensor-core kernel.
+constexpr int kChunk = 128;
 
 // Device scratch used by one forward call.
 struct Scratch {
-  float* qbar;     // [bH, N, d]  mean query per block, fp32
-  float* kbar;     // [bH, N, d]  mean key per block, fp32 (routing)
-  void* kbar_op;   // [bH, N, d]  mean key per block in the attention kernel's operand type
-  void* vbar_op;   // [bH, N, d]  V-hat_j / n_j in the attention kernel's operand type
-  uint32_t* mask;  // [bH, N, W]  bit j of row i: key block j selected for query block i
-  int32_t* counts; // [bH, N]     |S_i|
-  int32_t* tiles;  // [bH, N]     tiles of the attention loop: |S_i| + pooled-key chunks used
-  int32_t* order;  // [bH * N]    work items, head-major, heaviest first within a head
+  float* qbar;     // [bH, Nq, d]  mean query per block, fp32
+  float* kbar;     // [bH, Nk, d]  mean key per block, fp32 (routing)
+  void* kbar_op;   // [bH, Nk, d]  mean key per block in the attention kernel's operand type
+  void* vbar_op;   // [bH, Nk, d]  V-hat_j / n_j in the attention kernel's operand type
+  float* kvar;     // [bH, d]      Var_j(K-bar_j,c), population (diagonal sigma only)
+  uint32_t* mask;  // [bH, Nq, W]  bit j of row i: key block j selected for query block i
+  int32_t* counts; // [bH, Nq]     |S_i|
+  int32_t* tiles;  // [bH, Nq]     tiles of the attention loop: |S_i| + pooled-key chunks used
+  int32_t* order;  // [bH * Nq]    work items, head-major, heaviest first within a head
   int32_t* work_counter;  // 1 int, zeroed before the attention kernel
 };
 
 constexpr int kRouteMaxN = 40960;   // pooled keys per head the router handles
 constexpr int kOrderMaxN = 8192;    // query blocks per head the sorter handles
 
+// How sigma_i of Eq. 4 is estimated.
+enum SigmaMode : int {
+  kSigmaEq5 = 0,       // population std of the proxy-score row (Eq. 5)
+  kSigmaDiagonal = 1,  // scale * sqrt(sum_c Q-bar_ic^2 Var_j(K-bar_jc)): the diagonal estimator
+};
+
 // Prologue launches (prologue.cu).
 cudaError_t launch_pool(int in_dtype, int op_dtype, const void* q, const void* k, const void* v,
                         const Geometry& g, const Scratch& s, cudaStream_t st);
+// pair != 0: the attention kernel takes two selected key blocks per tile.
 cudaError_t launch_route(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
-                         cudaStream_t st);
+                         int sigma_mode, int pair, cudaStream_t st);
 cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st);
 
 // Attention launches.

@@ -7,7 +7,9 @@
 //   Eq. 4 / Eq. 5 -> route_kernel: the proxy row s_i = Q-bar_i K-bar^T / sqrt(d)
 //     is formed on chip (shared memory), its mean and population standard
 //     deviation give tau_i = mu_i + beta sigma_i, and S_i = {j : s_ij > tau_i}
-//     leaves as one bit per pair.  No N x N score map reaches global memory.
+//     leaves as one bit per pair.  No Nq x Nk score map reaches global memory.
+//     The diagonal estimator named beside Eq. 5 (kvar_kernel + route_kernel)
+//     takes sigma_i from the per-channel variances of K-bar instead.
 // All reductions run in a fixed order, so results are deterministic.
 #include <cmath>
 #include <cstdint>
@@ -70,49 +72,99 @@ __device__ void block_column_sums(const T* __restrict__ X, int n, float* __restr
   __syncthreads();
 }
 
-// grid (N, bH).  Q-bar (fp32), K-bar (fp32 and operand type), V-hat/n (operand type).
+// grid (max(Nq, Nk), bH).  CTA x pools query block x (Q-bar, fp32) if x < Nq
+// and key block x (K-bar in fp32 and in the operand type, V-hat/n in the
+// operand type) if x < Nk.
 template <typename T, typename Op, int D>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                            const T* __restrict__ v, int L, int B, int N,
-                                                            float* __restrict__ qbar, float* __restrict__ kbar,
-                                                            Op* __restrict__ kbar_op, Op* __restrict__ vbar_op) {
+                                                            const T* __restrict__ v, int L, int Bq, int Nq,
+                                                            int Bk, int Nk, float* __restrict__ qbar,
+                                                            float* __restrict__ kbar, Op* __restrict__ kbar_op,
+                                                            Op* __restrict__ vbar_op) {
   constexpr int VEC = 16 / sizeof(T);
   constexpr int R = kPoolThreads / (D / VEC);
   __shared__ float red[R * D];
   __shared__ float sums[D];
   const int blk = blockIdx.x, bh = blockIdx.y;
-  const int r0 = blk * B;
-  const int n = min(B, L - r0);
-  const float inv_n = 1.0f / (float)n;
-  const size_t head = (size_t)bh * L * D + (size_t)r0 * D;
-  const size_t prow = ((size_t)bh * N + blk) * D;
+  const size_t head = (size_t)bh * L * D;
 
-  block_column_sums<T, D>(q + head, n, red, sums);
-  for (int c = threadIdx.x; c < D; c += kPoolThreads) qbar[prow + c] = sums[c] * inv_n;
-  block_column_sums<T, D>(k + head, n, red, sums);
-  for (int c = threadIdx.x; c < D; c += kPoolThreads) {
-    float m = sums[c] * inv_n;
-    kbar[prow + c] = m;
-    if (kbar_op) kbar_op[prow + c] = from_f<Op>(m);
+  if (blk < Nq) {
+    const int r0 = blk * Bq;
+    const float inv_n = 1.0f / (float)min(Bq, L - r0);
+    block_column_sums<T, D>(q + head + (size_t)r0 * D, min(Bq, L - r0), red, sums);
+    const size_t prow = ((size_t)bh * Nq + blk) * D;
+    for (int c = threadIdx.x; c < D; c += kPoolThreads) qbar[prow + c] = sums[c] * inv_n;
   }
-  if (v != nullptr) {
-    block_column_sums<T, D>(v + head, n, red, sums);
-    for (int c = threadIdx.x; c < D; c += kPoolThreads) vbar_op[prow + c] = from_f<Op>(sums[c] * inv_n);
+  if (blk < Nk) {
+    const int r0 = blk * Bk;
+    const int n = min(Bk, L - r0);
+    const float inv_n = 1.0f / (float)n;
+    const size_t prow = ((size_t)bh * Nk + blk) * D;
+    block_column_sums<T, D>(k + head + (size_t)r0 * D, n, red, sums);
+    for (int c = threadIdx.x; c < D; c += kPoolThreads) {
+      float m = sums[c] * inv_n;
+      kbar[prow + c] = m;
+      if (kbar_op) kbar_op[prow + c] = from_f<Op>(m);
+    }
+    if (v != nullptr) {
+      block_column_sums<T, D>(v + head + (size_t)r0 * D, n, red, sums);
+      for (int c = threadIdx.x; c < D; c += kPoolThreads) vbar_op[prow + c] = from_f<Op>(sums[c] * inv_n);
+    }
+  }
+}
+
+// grid (bH), 256 threads.  kvar[bh, c] = population variance over the Nk key
+// blocks of K-bar_{j,c}, two passes (mean, then mean squared deviation); the
+// per-thread partial sums are added in a fixed order.
+template <int D>
+__global__ void __launch_bounds__(256) kvar_kernel(const float* __restrict__ kbar, int Nk,
+                                                   float* __restrict__ kvar) {
+  constexpr int R = 256 / D;
+  __shared__ float red[256];
+  __shared__ float mean_s[D];
+  const int bh = blockIdx.x, c = threadIdx.x % D, rl = threadIdx.x / D;
+  const float* kb = kbar + (size_t)bh * Nk * D;
+  float a = 0.f;
+  for (int j = rl; j < Nk; j += R) a += kb[(size_t)j * D + c];
+  red[threadIdx.x] = a;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float t = 0.f;
+    for (int r = 0; r < R; ++r) t += red[r * D + c];
+    mean_s[c] = t / (float)Nk;
+  }
+  __syncthreads();
+  const float m = mean_s[c];
+  float v = 0.f;
+  for (int j = rl; j < Nk; j += R) {
+    const float t = kb[(size_t)j * D + c] - m;
+    v = fmaf(t, t, v);
+  }
+  red[threadIdx.x] = v;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float t = 0.f;
+    for (int r = 0; r < R; ++r) t += red[r * D + c];
+    kvar[(size_t)bh * D + c] = t / (float)Nk;
   }
 }
 
 constexpr int kRouteThreads = 256;
 constexpr int kRouteKC = 32;  // pooled keys staged in shared memory at a time
 
-// grid (ceil(N / QB), bH), 256 threads, QB a multiple of 8 (up to 32).
+// grid (ceil(Nq / QB), bH), 256 threads, QB a multiple of 8 (up to 32).
 // Score pass: lane l takes staged key l, warp w the query blocks
 // w*QB/8 .. (w+1)*QB/8 - 1, so each thread runs QB/8 independent dot
 // products over one key row.  Row pass: warp w takes query blocks w, w + 8, ...
+// kvar == nullptr: sigma_i from the row (Eq. 5); else the diagonal estimator.
+// tiles[i] counts the attention kernel's tiles: pooled-key chunks used plus the
+// selected blocks, two to a tile when pair != 0.
 template <int D, int QPW>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __restrict__ qbar,
-                                                              const float* __restrict__ kbar, int N, int W,
-                                                              int B, int nchunk, float scale, float beta,
-                                                              int beta_mode, int correction,
+                                                              const float* __restrict__ kbar,
+                                                              const float* __restrict__ kvar, int Nq, int Nk,
+                                                              int W, int nchunk, float scale, float beta,
+                                                              int beta_mode, int correction, int pair,
                                                               uint32_t* __restrict__ mask,
                                                               int32_t* __restrict__ counts,
                                                               int32_t* __restrict__ tiles) {
@@ -120,17 +172,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
   extern __shared__ float sm[];
   float* qs = sm;                          // [QB][D]
   float* ks = qs + QB * D;                 // [KC][D + 1]
-  float* srow = ks + kRouteKC * (D + 1);   // [QB][N]
+  float* srow = ks + kRouteKC * (D + 1);   // [QB][Nk]
   const int bh = blockIdx.y;
   const int i0 = blockIdx.x * QB;
-  const int nq = min(QB, N - i0);
+  const int nq = min(QB, Nq - i0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const float* qb = qbar + ((size_t)bh * N + i0) * D;
-  const float* kb = kbar + (size_t)bh * N * D;
+  const float* qb = qbar + ((size_t)bh * Nq + i0) * D;
+  const float* kb = kbar + (size_t)bh * Nk * D;
 
   for (int e = tid; e < QB * D; e += kRouteThreads) qs[e] = e < nq * D ? qb[e] : 0.f;
-  for (int j0 = 0; j0 < N; j0 += kRouteKC) {
-    const int nk = min(kRouteKC, N - j0);
+  for (int j0 = 0; j0 < Nk; j0 += kRouteKC) {
+    const int nk = min(kRouteKC, Nk - j0);
     __syncthreads();
     for (int e = tid; e < nk * D; e += kRouteThreads) {
       int jj = e / D, c = e % D;
@@ -152,40 +204,46 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 #pragma unroll
       for (int q = 0; q < QPW; ++q) {
         const int qi = warp * QPW + q;
-        if (qi < nq) srow[(size_t)qi * N + j0 + lane] = acc[q] * scale;
+        if (qi < nq) srow[(size_t)qi * Nk + j0 + lane] = acc[q] * scale;
       }
     }
   }
   __syncthreads();
 
   for (int qi = warp; qi < nq; qi += kRouteThreads / 32) {
-    const float* s = srow + (size_t)qi * N;
+    const float* s = srow + (size_t)qi * Nk;
     // mean and population variance, two passes, lane-strided then a fixed tree
     float a = 0.f;
-    for (int j = lane; j < N; j += 32) a += s[j];
+    for (int j = lane; j < Nk; j += 32) a += s[j];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    const float mu = a / (float)N;
+    const float mu = a / (float)Nk;
     float v = 0.f;
-    for (int j = lane; j < N; j += 32) {
-      float t = s[j] - mu;
-      v = fmaf(t, t, v);
+    if (kvar == nullptr) {
+      for (int j = lane; j < Nk; j += 32) {
+        float t = s[j] - mu;
+        v = fmaf(t, t, v);
+      }
+    } else {
+      const float* qv = qs + qi * D;
+      const float* kvh = kvar + (size_t)bh * D;
+      for (int c = lane; c < D; c += 32) v = fmaf(qv[c] * qv[c], kvh[c], v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    const float sigma = sqrtf(v / (float)N);
+    const float sigma = kvar == nullptr ? sqrtf(v / (float)Nk) : scale * sqrtf(v);
     float tau;
     if (beta_mode < 0) tau = -INFINITY;
     else if (beta_mode > 0) tau = INFINITY;
     else tau = fmaf(beta, sigma, mu);
 
-    const size_t item = (size_t)bh * N + i0 + qi;
+    const size_t item = (size_t)bh * Nq + i0 + qi;
     uint32_t* mrow = mask + item * W;
     int cnt = 0;
     for (int w = lane; w < W; w += 32) {
       uint32_t bits = 0;
       const int jb = w * 32;
-      const int nb = min(32, N - jb);
+      const int nb = min(32, Nk - jb);
       for (int b = 0; b < nb; ++b) bits |= (s[jb + b] > tau ? 1u : 0u) << b;
       mrow[w] = bits;
       cnt += __popc(bits);
@@ -195,14 +253,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     // pooled-key chunks holding at least one unselected block
     int used = 0;
     if (correction) {
-      const int wpc = B / 32;  // mask words per chunk
+      constexpr int wpc = kChunk / 32;  // mask words per chunk
       for (int c = lane; c < nchunk; c += 32) {
         bool any = false;
         for (int q = 0; q < wpc; ++q) {
           const int w = c * wpc + q;
           if (w >= W) break;
           const int jb = w * 32;
-          const int nb = min(32, N - jb);
+          const int nb = min(32, Nk - jb);
           const uint32_t valid = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
           // recompute from scores: the words above may belong to other lanes
           uint32_t bits = 0;
@@ -216,7 +274,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     }
     if (lane == 0) {
       counts[item] = cnt;
-      tiles[item] = cnt + used;
+      tiles[item] = (pair ? (cnt + 1) >> 1 : cnt) + used;
     }
   }
 }
@@ -265,13 +323,15 @@ __global__ void identity_order_kernel(int32_t* order, int n) {
 template <typename T, typename Op>
 cudaError_t pool_dispatch(const void* q, const void* k, const void* v, const Geometry& g, const Scratch& s,
                           cudaStream_t st) {
-  dim3 grid(g.N, g.bH);
+  dim3 grid(g.Nq > g.Nk ? g.Nq : g.Nk, g.bH);
   if (g.d == 128)
-    pool_kernel<T, Op, 128><<<grid, kPoolThreads, 0, st>>>(
-        (const T*)q, (const T*)k, (const T*)v, g.L, g.B, g.N, s.qbar, s.kbar, (Op*)s.kbar_op, (Op*)s.vbar_op);
+    pool_kernel<T, Op, 128><<<grid, kPoolThreads, 0, st>>>((const T*)q, (const T*)k, (const T*)v, g.L, g.Bq,
+                                                           g.Nq, g.Bk, g.Nk, s.qbar, s.kbar, (Op*)s.kbar_op,
+                                                           (Op*)s.vbar_op);
   else
-    pool_kernel<T, Op, 64><<<grid, kPoolThreads, 0, st>>>(
-        (const T*)q, (const T*)k, (const T*)v, g.L, g.B, g.N, s.qbar, s.kbar, (Op*)s.kbar_op, (Op*)s.vbar_op);
+    pool_kernel<T, Op, 64><<<grid, kPoolThreads, 0, st>>>((const T*)q, (const T*)k, (const T*)v, g.L, g.Bq,
+                                                          g.Nq, g.Bk, g.Nk, s.qbar, s.kbar, (Op*)s.kbar_op,
+                                                          (Op*)s.vbar_op);
   return cudaGetLastError();
 }
 
@@ -288,50 +348,62 @@ cudaError_t launch_pool(int in_dtype, int op_dtype, const void* q, const void* k
 
 // Query blocks per CTA (QB = 8 * QPW), bounded by the shared memory their
 // score rows take.
-static int route_qpw(int N) {
+static int route_qpw(int Nk) {
   int qpw = 4;
-  while (qpw > 1 && (size_t)8 * qpw * N * sizeof(float) > 160u * 1024u) qpw >>= 1;
+  while (qpw > 1 && (size_t)8 * qpw * Nk * sizeof(float) > 160u * 1024u) qpw >>= 1;
   return qpw;
 }
 
 template <int D, int QPW>
 static cudaError_t route_launch(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
-                                cudaStream_t st) {
+                                int pair, const float* kvar, cudaStream_t st) {
   constexpr int QB = 8 * QPW;
-  const size_t smem = (size_t)(QB * D + kRouteKC * (D + 1) + (size_t)QB * g.N) * sizeof(float);
+  const size_t smem = (size_t)(QB * D + kRouteKC * (D + 1) + (size_t)QB * g.Nk) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(route_kernel<D, QPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((g.N + QB - 1) / QB, g.bH);
-  route_kernel<D, QPW><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, g.N, g.W, g.B, g.nchunk,
+  dim3 grid((g.Nq + QB - 1) / QB, g.bH);
+  route_kernel<D, QPW><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, g.W, g.nchunk,
                                                           1.0f / sqrtf((float)D), beta, beta_mode, correction,
-                                                          s.mask, s.counts, s.tiles);
+                                                          pair, s.mask, s.counts, s.tiles);
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t route_dispatch(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
+                                 int pair, const float* kvar, cudaStream_t st) {
+  const int qpw = route_qpw(g.Nk);
+  if (qpw == 4) return route_launch<D, 4>(g, s, beta, beta_mode, correction, pair, kvar, st);
+  if (qpw == 2) return route_launch<D, 2>(g, s, beta, beta_mode, correction, pair, kvar, st);
+  return route_launch<D, 1>(g, s, beta, beta_mode, correction, pair, kvar, st);
+}
+
 cudaError_t launch_route(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
-                         cudaStream_t st) {
-  const int qpw = route_qpw(g.N);
-  if (g.d == 128) {
-    if (qpw == 4) return route_launch<128, 4>(g, s, beta, beta_mode, correction, st);
-    if (qpw == 2) return route_launch<128, 2>(g, s, beta, beta_mode, correction, st);
-    return route_launch<128, 1>(g, s, beta, beta_mode, correction, st);
+                         int sigma_mode, int pair, cudaStream_t st) {
+  const float* kvar = nullptr;
+  if (sigma_mode == kSigmaDiagonal) {
+    if (g.d == 128)
+      kvar_kernel<128><<<g.bH, 256, 0, st>>>(s.kbar, g.Nk, s.kvar);
+    else
+      kvar_kernel<64><<<g.bH, 256, 0, st>>>(s.kbar, g.Nk, s.kvar);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    kvar = s.kvar;
   }
-  if (qpw == 4) return route_launch<64, 4>(g, s, beta, beta_mode, correction, st);
-  if (qpw == 2) return route_launch<64, 2>(g, s, beta, beta_mode, correction, st);
-  return route_launch<64, 1>(g, s, beta, beta_mode, correction, st);
+  if (g.d == 128) return route_dispatch<128>(g, s, beta, beta_mode, correction, pair, kvar, st);
+  return route_dispatch<64>(g, s, beta, beta_mode, correction, pair, kvar, st);
 }
 
 cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st) {
-  if (g.N > kOrderMaxN) {
+  if (g.Nq > kOrderMaxN) {
     identity_order_kernel<<<148, 256, 0, st>>>(s.order, g.nitems);
     return cudaGetLastError();
   }
   int P = 1;
-  while (P < g.N) P <<= 1;
+  while (P < g.Nq) P <<= 1;
   const size_t smem = (size_t)P * sizeof(unsigned long long);
   cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  order_kernel<<<g.bH, 1024, smem, st>>>(s.tiles, g.N, P, s.order);
+  order_kernel<<<g.bH, 1024, smem, st>>>(s.tiles, g.Nq, P, s.order);
   return cudaGetLastError();
 }
 
