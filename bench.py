@@ -252,8 +252,8 @@ def blocks_of(wl, args):
 
 
 def attention_kernel_name(wl, blk) -> str:
-    """The library runs tcgen05 for bf16, d = 128, Bq = 128, Bk in {64, 128}."""
-    tc = wl.dtype == torch.bfloat16 and wl.d == 128 and blk[0] == 128 and blk[1] in (64, 128)
+    """The library runs tcgen05 for bf16, d in {64, 128}, Bq = 128, Bk in {64, 128}."""
+    tc = wl.dtype == torch.bfloat16 and wl.d in (64, 128) and blk[0] == 128 and blk[1] in (64, 128)
     return "attn_tc_kernel" if tc else "attn_simt_kernel"
 
 

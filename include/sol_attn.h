@@ -74,9 +74,9 @@ typedef enum {
  * (independently: query blocks of Bq tokens, key blocks of Bk tokens, the
  * Eq. 9 weight of a key block is its token count); L >= 1; batch * heads >= 1;
  * batch * heads * L * d < 2^40; ceil(L / Bk) <= 40960; beta not NaN.
- * Other values return SOL_ERR_UNSUPPORTED.  bf16 with d == Bq == Bk == 128
- * runs the tensor-core (tcgen05/TMEM/TMA) kernel; every other supported
- * combination runs the CUDA-core kernel.
+ * Other values return SOL_ERR_UNSUPPORTED.  bf16 with Bq == 128 (any
+ * supported d and Bk) runs the tensor-core (tcgen05/TMEM/TMA) kernel; every
+ * other supported combination runs the CUDA-core kernel.
  */
 
 /*

@@ -176,10 +176,11 @@ def test_invalid_arguments_raise():
 # ------------------------------------------------------------------ workloads at full size
 
 @pytest.mark.parametrize("beta", [0.5, 1.04, 1.5])
-def test_image_dit(beta):
-    wl = I.WORKLOADS["image-dit"]
+@pytest.mark.parametrize("name,bk", [("image-dit", 128), ("image-dit-d64", 128), ("image-dit-d64", 64)])
+def test_image_dit(beta, name, bk):
+    wl = I.WORKLOADS[name]
     Q, K, V = I.make_workload(wl, device="cuda")
-    check_case(Q, K, V, wl.block, beta, sample_k=3, heads=range(wl.heads), seed=1)
+    check_case(Q, K, V, (wl.block, bk), beta, sample_k=3, heads=range(wl.heads), seed=1)
 
 
 @pytest.mark.parametrize("name,beta,bk", [("wan-480p", 1.04, 128),

@@ -108,10 +108,10 @@ cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
   return cudaMallocFromPoolAsync(p, bytes, pool, st);
 }
 
-// The tensor-core kernel is built for bf16 with d = 128, query blocks of 128
-// tokens and key blocks of 128 or 64 (two 64-token blocks share one tile).
+// The tensor-core kernel is built for bf16 with d in {64, 128}, query blocks
+// of 128 tokens and key blocks of 128 or 64 (two 64-token blocks share a tile).
 bool uses_tensor_cores(int dtype, const Geometry& g) {
-  return dtype == SOL_DTYPE_BF16 && g.d == 128 && g.Bq == 128 && (g.Bk == 128 || g.Bk == 64);
+  return dtype == SOL_DTYPE_BF16 && (g.d == 128 || g.d == 64) && g.Bq == 128 && (g.Bk == 128 || g.Bk == 64);
 }
 
 int pair_tiles(bool use_tc, const Geometry& g) { return use_tc && g.Bk == 64 ? 1 : 0; }

@@ -50,20 +50,31 @@ __device__ int g_sol_status;  // 0 = ok; else 0x1000 | wait id (first expiry)
 
 namespace {
 
-constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int QST = 1, KVST = 3;  // Q buffers, K+V stages
+constexpr int BM = 128, BN = 128;
+constexpr int QST = 1;  // Q buffers
 constexpr int NTHREADS = 320;
 constexpr int SOFTMAX_WARPS = 8;
-constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB, two 64-column swizzled halves
-constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_KV = OFF_Q + QST * TILE_BYTES;  // stage s: K at +2s tiles, V at +2s+1
-constexpr uint32_t OFF_BAR = OFF_KV + 2 * KVST * TILE_BYTES;  // 224 KB
+constexpr uint32_t SLAB = BM * 128;  // 16 KB: 64 bf16 columns of a 128-row tile, 128-byte swizzled
 constexpr uint32_t BAR_AREA = 2560;
-// No room for alignment slack: the kernel checks that dynamic shared memory
-// starts on a 1024-byte boundary (the 128-byte swizzle needs it) and reports
-// an error instead of running if it does not.
-constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA;
+
+// Shared-memory plan for head dimension HD (64 or 128).  A Q, K or V tile is
+// HD / 64 slabs; the K+V ring gets as many stages as fit (3 at d = 128, 6 at
+// d = 64).  There is no room for alignment slack: the kernel checks that
+// dynamic shared memory starts on a 1024-byte boundary (the 128-byte swizzle
+// needs it) and reports an error instead of running if it does not.
+template <int HD>
+struct Cfg {
+  static_assert(HD == 64 || HD == 128, "head dimension");
+  static constexpr int NSLAB = HD / 64;
+  static constexpr uint32_t TILE_BYTES = NSLAB * SLAB;
+  static constexpr int KVST = HD == 128 ? 3 : 6;  // K+V stages
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_KV = OFF_Q + QST * TILE_BYTES;  // stage s: K at +2s tiles, V at +2s+1
+  static constexpr uint32_t OFF_BAR = OFF_KV + 2 * KVST * TILE_BYTES;
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA;
+  static constexpr int OCHUNK = HD / 64;  // 32-column output chunks per softmax half
+};
+static_assert(Cfg<128>::SMEM_BYTES <= 227 * 1024 && Cfg<64>::SMEM_BYTES <= 227 * 1024, "shared memory");
 
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_P = 384;  // O_h at TM_O + 128 h
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -91,6 +102,7 @@ struct Params {
   int chunks;           // pooled-key chunks walked per item: nchunk, or 0 without the correction
 };
 
+template <int KVST>
 struct Bars {
   uint64_t q_full[QST], q_empty[QST];
   uint64_t kv_full[KVST], kv_empty[KVST];
@@ -108,7 +120,8 @@ struct Bars {
   float xm[2][BM];        // [column half][row] running max (log2 units)
   float xl[2][BM];        // [column half][row] row sum
 };
-static_assert(sizeof(Bars) <= BAR_AREA, "barrier area");
+static_assert(sizeof(Bars<Cfg<64>::KVST>) <= BAR_AREA && sizeof(Bars<Cfg<128>::KVST>) <= BAR_AREA,
+              "barrier area");
 static_assert(QST == 1, "one Q buffer");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
@@ -161,7 +174,8 @@ struct TileIter {
 
 // All 32 lanes wait; the outcome is made warp-uniform so that warp-wide
 // instructions that follow are never reached by part of a warp.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Bars& B_, uint64_t lim, int id) {
+template <class BarsT>
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, BarsT& B_, uint64_t lim, int id) {
   const bool ok = mbar_wait(bar, parity, &B_.abort_flag, &g_sol_status, 0x1000 | id, lim);
   return __all_sync(0xffffffffu, ok);
 }
@@ -200,17 +214,22 @@ __device__ __forceinline__ float tree_max64(const float (&x)[64]) {
   return max3(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
 }
 
+template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                    const __grid_constant__ CUtensorMap tmVb, const Params p) {
+  using C = Cfg<HD>;
+  constexpr int KVST = C::KVST;
+  constexpr int NSLAB = C::NSLAB;
+  constexpr uint32_t TILE_BYTES = C::TILE_BYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {
     if (threadIdx.x == 0) atomicCAS(&g_sol_status, 0, 0x2000);
     return;
   }
   uint8_t* smem = smem_raw;
-  Bars& bars = *reinterpret_cast<Bars*>(smem + OFF_BAR);
+  Bars<KVST>& bars = *reinterpret_cast<Bars<KVST>*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.wait_limit_ns;
 
@@ -278,9 +297,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (qu > 0 && !(ok = wait_warp(&bars.q_empty[qb], (qu - 1) & 1, bars, lim, 2))) break;
       if (leader) {
         mbar_arrive_expect_tx(&bars.q_full[qb], TILE_BYTES);
-        uint8_t* qdst = smem + OFF_Q + qb * TILE_BYTES;
-        tma_load_3d(qdst, &tmQ, &bars.q_full[qb], 0, qi * BM, bh, pol_q);
-        tma_load_3d(qdst + HALF_BYTES, &tmQ, &bars.q_full[qb], 64, qi * BM, bh, pol_q);
+        uint8_t* qdst = smem + C::OFF_Q + qb * TILE_BYTES;
+#pragma unroll
+        for (int hd = 0; hd < NSLAB; ++hd)
+          tma_load_3d(qdst + hd * SLAB, &tmQ, &bars.q_full[qb], hd * 64, qi * BM, bh, pol_q);
       }
       ++q_uses;
       TileIter ti;
@@ -294,7 +314,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // stage ks is free once the PV of its previous tile has finished
         if (ku > 0 && !(ok = wait_warp(&bars.kv_empty[ks], (ku - 1) & 1, bars, lim, 3))) break;
         if (leader) {
-          uint8_t* dk = smem + OFF_KV + (2 * ks) * TILE_BYTES;
+          uint8_t* dk = smem + C::OFF_KV + (2 * ks) * TILE_BYTES;
           uint8_t* dv = dk + TILE_BYTES;
           mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
           if (kind == 1 && p.pair) {
@@ -302,19 +322,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // a tile with one block repeats it in the second half (masked out)
             const int j2 = tidx2 >= 0 ? tidx2 : tidx;
 #pragma unroll
-            for (int hd = 0; hd < 2; ++hd) {
-              tma_load_3d(dk + hd * HALF_BYTES, &tmK, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
-              tma_load_3d(dk + hd * HALF_BYTES + 64 * 128, &tmK, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
-              tma_load_3d(dv + hd * HALF_BYTES, &tmV, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
-              tma_load_3d(dv + hd * HALF_BYTES + 64 * 128, &tmV, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+            for (int hd = 0; hd < NSLAB; ++hd) {
+              tma_load_3d(dk + hd * SLAB, &tmK, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+              tma_load_3d(dk + hd * SLAB + 64 * 128, &tmK, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+              tma_load_3d(dv + hd * SLAB, &tmV, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+              tma_load_3d(dv + hd * SLAB + 64 * 128, &tmV, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
             }
           } else {
             const CUtensorMap* mk = kind ? &tmK : &tmKb;
             const CUtensorMap* mv = kind ? &tmV : &tmVb;
-            tma_load_3d(dk, mk, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
-            tma_load_3d(dk + HALF_BYTES, mk, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
-            tma_load_3d(dv, mv, &bars.kv_full[ks], 0, tidx * BN, bh, pol_kv);
-            tma_load_3d(dv + HALF_BYTES, mv, &bars.kv_full[ks], 64, tidx * BN, bh, pol_kv);
+#pragma unroll
+            for (int hd = 0; hd < NSLAB; ++hd) {
+              tma_load_3d(dk + hd * SLAB, mk, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
+              tma_load_3d(dv + hd * SLAB, mv, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
+            }
           }
         }
         gk_last = (int)gk;
@@ -337,7 +358,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const bool leader = elect_one();
     constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-    const uint32_t sKV = smem_u32(smem + OFF_KV);
+    const uint32_t sKV = smem_u32(smem + C::OFF_KV);
     uint32_t g = 0;
     int item_local = 0;  // items with T > 0 processed
     bool issued = false;
@@ -352,7 +373,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          const uint32_t off = (kk >> 2) * SLAB + (kk & 3) * 32;
           mma_ss(tmem + TM_S, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
                  IDESC_QK, kk > 0 ? 1u : 0u);
         }
@@ -375,7 +396,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + TM_O + h * 128, tmem + TM_P + pb * 64 + h * 32 + kk * 8,
-                   smem_desc_sw128(vbase + h * 8192 + kk * 2048, HALF_BYTES, 1024), IDESC_PV,
+                   smem_desc_sw128(vbase + h * 8192 + kk * 2048, SLAB, 1024), IDESC_PV,
                    (first && kk == 0) ? 0u : 1u);
         }
         tc_commit(&bars.kv_empty[ks]);
@@ -395,7 +416,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (T == 0) continue;
       const int qb = item_local % QST;
       if (!(ok = wait_warp(&bars.q_full[qb], (item_local / QST) & 1, bars, lim, 11))) break;
-      const uint32_t sQ = smem_u32(smem + OFF_Q + qb * TILE_BYTES);
+      const uint32_t sQ = smem_u32(smem + C::OFF_Q + qb * TILE_BYTES);
       // order: S_0, then for each tile n: S_{n+1}, PV_n
       if (!(ok = issue_s(g, sQ))) break;
       issued = true;
@@ -425,7 +446,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int half = (warp - 2) >> 2;     // column half of every S tile this warp owns
     const int quad = warp & 3;            // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;     // query row within the tile
-    const int col0 = half * 64;
+    const int col0 = half * 64;        // this half's key columns of an S tile
+    const int ocol0 = half * (HD / 2);  // this half's output columns
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tO = tmem + lane_off + TM_O + half * 128;  // this half's accumulator O_h
     const float sl2 = p.scale_log2;
@@ -442,10 +464,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int bh = item / p.Nq, qi = item % p.Nq;
       const int T = p.tiles[item];
       const int n_rows = min(BM, p.L - qi * BM);
-      __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD + col0;
+      __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD + ocol0;
       if (T == 0) {
         if (row < n_rows)
-          for (int c = 0; c < 64; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < HD / 2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
       TileIter ti;
@@ -565,7 +587,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!(ok = wait_warp(&bars.pv_done[gp & 1], (gp >> 1) & 1, bars, lim, 23))) break;
           tc_fence_after();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < HD / 32; ++q) {
             uint32_t o[32];
             tmem_ld32(tO + q * 32, o);
             tmem_wait_ld();
@@ -592,11 +614,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) mbar_arrive(&bars.xstate);
       if (!(ok = wait_warp(&bars.o_full, item_local & 1, bars, lim, 24))) break;
       tc_fence_after();
-      uint32_t o0[2][32], o1[2][32];
-      tmem_ld32(tmem + lane_off + TM_O + col0, o0[0]);
-      tmem_ld32(tmem + lane_off + TM_O + col0 + 32, o0[1]);
-      tmem_ld32(tmem + lane_off + TM_O + 128 + col0, o1[0]);
-      tmem_ld32(tmem + lane_off + TM_O + 128 + col0 + 32, o1[1]);
+      constexpr int OCH = C::OCHUNK;
+      uint32_t o0[OCH][32], o1[OCH][32];
+#pragma unroll
+      for (int q = 0; q < OCH; ++q) {
+        tmem_ld32(tmem + lane_off + TM_O + ocol0 + q * 32, o0[q]);
+        tmem_ld32(tmem + lane_off + TM_O + 128 + ocol0 + q * 32, o1[q]);
+      }
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -612,7 +636,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float w0 = e0 * inv, w1 = e1 * inv;
       if (row < n_rows) {
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < OCH; ++q) {
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
             float v[8];
@@ -658,9 +682,9 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [planes, rows, 128] bf16 tensor, boxes of 64 columns x box_rows rows,
+// [planes, rows, HD] bf16 tensor, boxes of 64 columns x box_rows rows,
 // 128-byte swizzle; rows past `rows` read as zero.
-bool make_map(CUtensorMap* m, const void* base, int rows, int planes, int box_rows) {
+bool make_map(CUtensorMap* m, const void* base, int HD, int rows, int planes, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)rows, (cuuint64_t)planes};
@@ -672,16 +696,32 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int planes, int box_ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int HD>
+cudaError_t launch_hd(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtensorMap& mV, const CUtensorMap& mKb,
+                      const CUtensorMap& mVb, const Params& p, int nitems, cudaStream_t st) {
+  constexpr uint32_t smem = Cfg<HD>::SMEM_BYTES;
+  int dev = 0, nsm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = nitems < nsm ? nitems : nsm;
+  attn_tc_kernel<HD><<<grid, NTHREADS, smem, st>>>(mQ, mK, mV, mKb, mVb, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
                            const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction) {
   CUtensorMap mQ, mK, mV, mKb, mVb;
-  // built for d == 128, query blocks of 128 tokens, key blocks of 128 or 64
-  if (g.Bq != BM || (g.Bk != BN && g.Bk != BN / 2) || g.d != HD) return cudaErrorInvalidValue;
-  if (!make_map(&mQ, q, g.L, g.bH, BM) || !make_map(&mK, k, g.L, g.bH, g.Bk) ||
-      !make_map(&mV, v, g.L, g.bH, g.Bk) || !make_map(&mKb, s.kbar_op, g.Nk, g.bH, BN) ||
-      !make_map(&mVb, s.vbar_op, g.Nk, g.bH, BN))
+  // built for d in {64, 128}, query blocks of 128 tokens, key blocks of 128 or 64
+  if (g.Bq != BM || (g.Bk != BN && g.Bk != BN / 2) || (g.d != 64 && g.d != 128)) return cudaErrorInvalidValue;
+  if (!make_map(&mQ, q, g.d, g.L, g.bH, BM) || !make_map(&mK, k, g.d, g.L, g.bH, g.Bk) ||
+      !make_map(&mV, v, g.d, g.L, g.bH, g.Bk) || !make_map(&mKb, s.kbar_op, g.d, g.Nk, g.bH, BN) ||
+      !make_map(&mVb, s.vbar_op, g.d, g.Nk, g.bH, BN))
     return cudaErrorInvalidValue;
   Params p;
   p.bH = g.bH; p.L = g.L; p.Nq = g.Nq; p.Nk = g.Nk; p.W = g.W; p.nchunk = g.nchunk; p.nitems = g.nitems;
@@ -694,16 +734,8 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.out = static_cast<__nv_bfloat16*>(out);
   p.wait_limit_ns = wait_limit_ns;
   p.chunks = correction ? g.nchunk : 0;
-  int dev = 0, nsm = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const int grid = g.nitems < nsm ? g.nitems : nsm;
-  attn_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(mQ, mK, mV, mKb, mVb, p);
-  return cudaGetLastError();
+  if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+  return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
 }
 
 cudaError_t read_device_status(cudaStream_t st, int32_t* word) {

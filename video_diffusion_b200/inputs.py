@@ -77,6 +77,10 @@ WORKLOADS = {
     "hunyuan-720p": Workload(
         "HunyuanVideo-13B 720p (24 heads, L=118800+256 text on 33x45x80, d=128, B=128)",
         torch.bfloat16, 1, 24, 128, (33, 45, 80), 256, 128, (1.04, 1.5), 1004),
+    # image-DiT geometry with 64-wide heads (the head width of several image DiTs)
+    "image-dit-d64": Workload(
+        "image-DiT d=64 heads (24 heads, L=16384 on 1x128x128, d=64, B=128)",
+        torch.bfloat16, 1, 24, 64, (1, 128, 128), 0, 128, (0.5, 1.04, 1.5), 1005),
 }
 
 
