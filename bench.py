@@ -240,6 +240,8 @@ def config_of(wl, args):
         c["block_k"] = args.block_k
     if args.diagonal_sigma:
         c["sigma"] = "diagonal estimator"
+    if args.route_in_kernel:
+        c["routing"] = "inside the attention kernel"
     return c
 
 
@@ -372,6 +374,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block-k", type=int, default=None,
                     help="key block size (default: the workload's block size, the same as the query block)")
+    ap.add_argument("--route-in-kernel", action="store_true",
+                    help="let the attention kernel decide the selection itself (no selection mask)")
     ap.add_argument("--diagonal-sigma", action="store_true",
                     help="sigma_i of Eq. 4 from the diagonal moment estimator instead of Eq. 5")
     ap.add_argument("--sweep-beta", default=None,
@@ -416,7 +420,7 @@ def main():
     del sel, counts
 
     for _ in range(args.warmup):
-        api.forward_ex(Q, K, V, args.beta, blk, out=out, diagonal_sigma=diag)
+        api.forward_ex(Q, K, V, args.beta, blk, out=out, diagonal_sigma=diag, route_in_kernel=args.route_in_kernel)
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -430,7 +434,8 @@ def main():
         clocks.mark_start()
         start.record(stream)
         for s in range(args.steps):
-            api.forward_ex(Q, K, V, args.beta, blk, out=out, events=evs[s], diagonal_sigma=diag)
+            api.forward_ex(Q, K, V, args.beta, blk, out=out, events=evs[s], diagonal_sigma=diag,
+                           route_in_kernel=args.route_in_kernel)
         end.record(stream)
         torch.cuda.synchronize()
         clocks.mark_end()
@@ -473,7 +478,8 @@ def main():
             dQ.copy_(hQ, non_blocking=True)
             dK.copy_(hK, non_blocking=True)
             dV.copy_(hV, non_blocking=True)
-            api.forward_ex(dQ, dK, dV, args.beta, blk, out=out, diagonal_sigma=diag)
+            api.forward_ex(dQ, dK, dV, args.beta, blk, out=out, diagonal_sigma=diag,
+                           route_in_kernel=args.route_in_kernel)
             hO.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()

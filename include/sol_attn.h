@@ -63,6 +63,13 @@ typedef enum {
                                      variance of each pooled-key channel over the key blocks,
                                      i.e. Eq. 5 with the off-diagonal covariance dropped).
                                      mu_i is unchanged. */
+#define SOL_FLAG_ROUTE_IN_KERNEL 4u /* Eq. 4 decided inside the tensor-core attention kernel
+                                     (the producer warp scores each key block from the fp32
+                                     pooled vectors with the router's arithmetic and compares
+                                     with the router's tau_i; Eq. 11's "proxy reuse"): no
+                                     selection mask is written or read.  Same results as
+                                     without the flag.  Tensor-core calls only (bf16, Bq = 128)
+                                     with ceil(L / Bk) <= 2048, else SOL_ERR_UNSUPPORTED. */
 
 typedef enum {
   SOL_DTYPE_BF16 = 0,           /* bfloat16 inputs and output; fp32 accumulation */
@@ -118,8 +125,8 @@ int sol_attn_stats_ex(const void* q, const void* k, int32_t* counts, uint32_t* m
 /*
  * Extended forward.  Arguments as sol_attn_forward plus:
  *   dtype  : sol_dtype of q, k, v, out
- *   flags  : 0 or an OR of SOL_FLAG_KEEP_OR_DROP, SOL_FLAG_DIAGONAL_SIGMA
- *            (unknown bits: SOL_ERR_INVALID_ARG)
+ *   flags  : 0 or an OR of SOL_FLAG_KEEP_OR_DROP, SOL_FLAG_DIAGONAL_SIGMA,
+ *            SOL_FLAG_ROUTE_IN_KERNEL (unknown bits: SOL_ERR_INVALID_ARG)
  *   events : NULL, or 4 cudaEvent_t the library records on `stream`
  *            before pooling, after pooling, after routing and after the
  *            attention kernel (time each stage with cudaEventElapsedTime)
@@ -160,7 +167,7 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
 /* Human-readable name of a sol_status value. */
 const char* sol_attn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor): 102. */
+/* Library ABI version (major * 100 + minor): 103. */
 int sol_attn_version(void);
 
 #ifdef __cplusplus

@@ -39,7 +39,7 @@ def test_status_strings_and_version(L):
     assert api.status_string(-1) == "SOL_ERR_INVALID_ARG"
     assert api.status_string(-5) == "SOL_ERR_DEVICE_TIMEOUT"
     assert api.status_string(7) == "SOL_ERR_UNKNOWN"
-    assert api.version() == 102
+    assert api.version() == 103
 
 
 # Argument checks run on the host before any CUDA call, so fake device
@@ -69,14 +69,19 @@ def test_stats_and_ex_reject_bad_arguments(L):
     assert L.sol_attn_stats(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 128, f(1.0), 9, None) == -1
     assert L.sol_attn_stats(FAKE, FAKE, FAKE, None, 1, 1, 256, 100, 128, 128, f(1.0), 0, None) == -2
     assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 5, 1, 1, 256, 128, 128, 128, f(1.0), 0, None, None) == -1
-    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 128, 128, f(1.0), 6, None, None) == -1
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 128, 128, f(1.0), 9, None, None) == -1
     assert L.sol_attn_forward_f32(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 64, 64, f(math.nan), None) == -1
     # stats_ex takes SOL_FLAG_DIAGONAL_SIGMA only; forward_ex both flags, no other bit
     assert L.sol_attn_stats_ex(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, 1, None) == -1
     assert L.sol_attn_stats_ex(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, 4, None) == -1
     assert L.sol_attn_stats_ex(FAKE, FAKE, None, None, 1, 1, 256, 128, 128, 128, f(1.0), 0, 2, None) == -1
     assert L.sol_attn_stats_ex(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 128, 96, f(1.0), 0, 2, None) == -2
-    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 128, 128, f(1.0), 4, None, None) == -1
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 128, 128, f(1.0), 8, None, None) == -1
+    # in-kernel routing: tensor-core calls only, at most 2048 key blocks
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 256, 128, 128, 128, f(1.0), 4, None, None) == -2
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 128, 64, 64, f(1.0), 4, None, None) == -2
+    assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 64 * 2049, 128, 128, 64, f(1.0), 4, None,
+                                 None) == -2
     assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 96, 128, 64, f(1.0), 3, None, None) == -2
 
 

@@ -256,3 +256,49 @@ def test_keep_or_drop_fp32(beta):
     wl = I.WORKLOADS["tiny-fp32"]
     Q, K, V = I.make_workload(wl, device="cuda")
     check_keep_or_drop(Q, K, V, wl.block, beta)
+
+
+# ------------------------------------------------------------------ routing inside the attention kernel
+
+@pytest.mark.parametrize("name,bk,beta", [("wan-480p", 128, 1.04), ("wan-480p", 64, 1.04), ("image-dit", 128, 0.5),
+                                          ("image-dit-d64", 128, 1.5), ("hunyuan-720p", 64, 1.04),
+                                          ("wan-720p", 128, -INF), ("wan-720p", 128, INF)])
+def test_route_in_kernel_is_bit_identical(name, bk, beta):
+    """The attention kernel's own Eq. 4 decisions (router arithmetic on the
+    fp32 pooled vectors) select exactly the router's blocks, so the output is
+    the same bits as with the router's mask."""
+    wl = I.WORKLOADS[name]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    a = api.forward_ex(Q, K, V, beta, (wl.block, bk))
+    b = api.forward_ex(Q, K, V, beta, (wl.block, bk), route_in_kernel=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("block", [128, (128, 64)])
+@pytest.mark.parametrize("beta", [-INF, 0.5, 1.04, INF])
+def test_route_in_kernel_against_oracle(block, beta):
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=14, device="cuda")  # ragged L = 1000
+    out = torch.full_like(Q, float("nan"))
+    api.forward_ex(Q, K, V, beta, block, out=out, route_in_kernel=True)
+    counts, sel = api.stats(Q, K, beta, block, with_mask=True)
+    torch.cuda.synchronize()
+    sel, counts = sel.cpu().numpy(), counts.cpu().numpy()
+    bq, bk = P.pair(block)
+    gpu_rows, ref_rows = [], []
+    for h in range(2):
+        r = O.route_head(P.head_np(Q, 0, h), P.head_np(K, 0, h), bq, bk, beta)
+        P.compare_selection(r, sel[0, h], counts[0, h])
+        ref_rows.append(P.oracle_rows(Q, K, V, 0, h, block, beta, sel[0, h], list(range(r["qgeom"].n))))
+        gpu_rows.append(out[0, h].double().cpu().numpy())
+    assert not torch.isnan(out).any()
+    P.check_close(np.concatenate(gpu_rows), np.concatenate(ref_rows), torch.bfloat16, "route in kernel")
+
+
+def test_route_in_kernel_with_keep_or_drop_and_diagonal_sigma():
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=15, device="cuda")
+    for kw in (dict(keep_or_drop=True), dict(diagonal_sigma=True), dict(keep_or_drop=True, diagonal_sigma=True)):
+        a = api.forward_ex(Q, K, V, 1.04, 128, **kw)
+        b = api.forward_ex(Q, K, V, 1.04, 128, route_in_kernel=True, **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b), kw

@@ -22,6 +22,7 @@ STATUS = {0: "SOL_OK", -1: "SOL_ERR_INVALID_ARG", -2: "SOL_ERR_UNSUPPORTED", -3:
 DTYPE_BF16, DTYPE_F32 = 0, 1
 FLAG_KEEP_OR_DROP = 1  # correction off: unselected blocks contribute nothing
 FLAG_DIAGONAL_SIGMA = 2  # sigma_i from the diagonal moment estimator
+FLAG_ROUTE_IN_KERNEL = 4  # Eq. 4 decided inside the attention kernel (no selection mask)
 
 EXPORTS = ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
            "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_status_string", "sol_attn_version")
@@ -115,13 +116,15 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, bloc
 
 
 def forward_ex(q, k, v, beta: float, block=128, out=None, events=None, stream=None,
-               keep_or_drop: bool = False, diagonal_sigma: bool = False) -> torch.Tensor:
+               keep_or_drop: bool = False, diagonal_sigma: bool = False,
+               route_in_kernel: bool = False) -> torch.Tensor:
     """forward() that also records up to four torch.cuda.Event objects: before
     pooling, after pooling, after routing, after the attention kernel.  The
     events must exist already (torch creates them on their first record()).
     keep_or_drop=True switches the correction off (unselected blocks
     contribute nothing; rows with no selected block give 0); diagonal_sigma=True
-    takes sigma_i from the diagonal moment estimator."""
+    takes sigma_i from the diagonal moment estimator; route_in_kernel=True has
+    the attention kernel decide the selection itself (same results)."""
     b, h, L, d = _shape(q, k, v)
     bq, bk = blocks(block)
     if out is None:
@@ -137,7 +140,8 @@ def forward_ex(q, k, v, beta: float, block=128, out=None, events=None, stream=No
     rc = lib().sol_attn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
                                    b, h, L, d, bq, bk, float(beta),
                                    (FLAG_KEEP_OR_DROP if keep_or_drop else 0)
-                                   | (FLAG_DIAGONAL_SIGMA if diagonal_sigma else 0), ev, _stream_handle(stream))
+                                   | (FLAG_DIAGONAL_SIGMA if diagonal_sigma else 0)
+                                   | (FLAG_ROUTE_IN_KERNEL if route_in_kernel else 0), ev, _stream_handle(stream))
     _check("sol_attn_forward_ex", rc)
     return out
 

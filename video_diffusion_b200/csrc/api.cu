@@ -69,6 +69,7 @@ size_t carve(const Geometry& g, size_t op_elem, char* base, Scratch* s) {
   s->vbar_op = take(kpooled * op_elem);
   s->kvar = reinterpret_cast<float*>(take((size_t)g.bH * g.d * sizeof(float)));
   s->mask = reinterpret_cast<uint32_t*>(take((size_t)g.nitems * g.W * sizeof(uint32_t)));
+  s->tau = reinterpret_cast<float*>(take((size_t)g.nitems * sizeof(float)));
   s->counts = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
   s->tiles = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
   s->order = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
@@ -136,13 +137,16 @@ int record(void* const* events, int i, cudaStream_t st) {
 int forward_impl(const void* q, const void* k, const void* v, void* out, int dtype, int batch, int heads, int L,
                  int d, int Bq, int Bk, float beta, unsigned flags, void* const* events, cudaStream_t st) {
   if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
-  if (flags & ~(SOL_FLAG_KEEP_OR_DROP | SOL_FLAG_DIAGONAL_SIGMA)) return SOL_ERR_INVALID_ARG;
+  if (flags & ~(SOL_FLAG_KEEP_OR_DROP | SOL_FLAG_DIAGONAL_SIGMA | SOL_FLAG_ROUTE_IN_KERNEL))
+    return SOL_ERR_INVALID_ARG;
   const int correction = (flags & SOL_FLAG_KEEP_OR_DROP) ? 0 : 1;
   const int sigma_mode = (flags & SOL_FLAG_DIAGONAL_SIGMA) ? sol::kSigmaDiagonal : sol::kSigmaEq5;
+  const int inkernel = (flags & SOL_FLAG_ROUTE_IN_KERNEL) ? 1 : 0;
   Geometry g;
   int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
   if (rc != SOL_OK) return rc;
   const bool use_tc = uses_tensor_cores(dtype, g);
+  if (inkernel && (!use_tc || g.W > sol::kInKernelMaxW)) return SOL_ERR_UNSUPPORTED;
   const int op_dtype = use_tc ? 0 : 1;  // operand type of K-bar / V-bar: bf16 for tensor cores
   Scratch s;
   const size_t bytes = carve(g, use_tc ? 2 : 4, nullptr, &s);
@@ -152,6 +156,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
     return SOL_ERR_NO_MEMORY;
   }
   carve(g, use_tc ? 2 : 4, static_cast<char*>(base), &s);
+  if (inkernel) s.mask = nullptr;  // no decision record: the attention kernel decides
   cudaError_t e = cudaSuccess;
   const int in_dtype = dtype == SOL_DTYPE_BF16 ? 0 : 1;
   if ((rc = record(events, 0, st)) != SOL_OK) goto done;
@@ -166,7 +171,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   if (use_tc) {
     e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) goto done;
-    e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), correction);
+    e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), correction, inkernel);
   } else {
     e = sol::launch_attn_simt(in_dtype, q, k, v, out, g, s, st, correction);
   }
@@ -252,7 +257,7 @@ const char* sol_attn_status_string(int status) {
   }
 }
 
-int sol_attn_version(void) { return 102; }
+int sol_attn_version(void) { return 103; }
 
 }  // extern "C"
 
@@ -322,7 +327,7 @@ extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void
   if (e == cudaSuccess) e = sol::launch_order(g, s, st);
   if (use_tc) {
     if (e == cudaSuccess) e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
-    if (e == cudaSuccess) e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), 1);
+    if (e == cudaSuccess) e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), 1, 0);
   } else if (e == cudaSuccess) {
     e = sol::launch_attn_simt(0, q, k, v, out, g, s, st, 1);
   }

@@ -33,12 +33,15 @@
 //               max, row sum and fp32 accumulator O_h = sum P_h V_h, so the
 //               halves never wait for each other inside the key loop; the two
 //               partial softmax states of a row are merged once per item.
-// TMEM columns: S [0,128), O_0 [128,256), O_1 [256,384), P [384,512) as two
-// buffers of 64 columns, each holding half 0's then half 1's 64 bf16 pairs.
+// TMEM columns: two S buffers [0,128) and [128,256) (tile n in buffer n % 2,
+// so S of the next tile is computed while the softmax works on this one; the
+// softmax writes P as bf16 pairs over the first 32 columns of each 64-column
+// half of its S), O_0 [256,384), O_1 [384,512).
 // Every mbarrier wait is bounded; on expiry the CTA abandons its work, waits
 // for its own copies and MMAs, frees TMEM and records the failing wait in the
 // device status word.
 #include <cmath>
+#include <cstddef>
 #include <cstdint>
 
 #include "common.cuh"
@@ -55,7 +58,7 @@ constexpr int QST = 1;  // Q buffers
 constexpr int NTHREADS = 320;
 constexpr int SOFTMAX_WARPS = 8;
 constexpr uint32_t SLAB = BM * 128;  // 16 KB: 64 bf16 columns of a 128-row tile, 128-byte swizzled
-constexpr uint32_t BAR_AREA = 2560;
+constexpr uint32_t BAR_AREA = 3072;
 
 // Shared-memory plan for head dimension HD (64 or 128).  A Q, K or V tile is
 // HD / 64 slabs; the K+V ring gets as many stages as fit (3 at d = 128, 6 at
@@ -76,7 +79,10 @@ struct Cfg {
 };
 static_assert(Cfg<128>::SMEM_BYTES <= 227 * 1024 && Cfg<64>::SMEM_BYTES <= 227 * 1024, "shared memory");
 
-constexpr uint32_t TM_S = 0, TM_O = 128, TM_P = 384;  // O_h at TM_O + 128 h
+// TMEM columns: S buffer b at TM_S + 128 b (tile gs uses buffer gs % 2; its
+// P overwrites the first 32 columns of each 64-column half, as bf16 pairs),
+// O_h at TM_O + 128 h
+constexpr uint32_t TM_S = 0, TM_O = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 // Column pairs p with (p % 8) in {2, 5, 7} (3 of 8, 24 of a thread's 64
@@ -100,21 +106,40 @@ struct Params {
   __nv_bfloat16* out;
   uint64_t wait_limit_ns;
   int chunks;           // pooled-key chunks walked per item: nchunk, or 0 without the correction
+  // routing inside the kernel (route_inkernel != 0): the producer warp decides
+  // S_i from the fp32 pooled vectors and the router's tau_i instead of reading
+  // the mask; the arithmetic is the router's, so the sets are identical
+  int route_inkernel;
+  float scale;          // 1/sqrt(d) as the router computes it
+  const float* qbar;    // [bH, Nq, d] fp32
+  const float* kbar;    // [bH, Nk, d] fp32
+  const float* tau;     // [bH * Nq]
+};
+
+// What the producer tells the other roles about the tile in one ring stage:
+// kind 0 = pooled chunk idx (vm: its unselected, in-range pooled keys, 4
+// words), kind 1 = exact key block idx (and idx2 for a 64-token pair, or -1).
+struct TileDesc {
+  int kind, idx, idx2;
+  uint32_t vm[4];
 };
 
 template <int KVST>
 struct Bars {
   uint64_t q_full[QST], q_empty[QST];
   uint64_t kv_full[KVST], kv_empty[KVST];
-  uint64_t s_full, s_free;
-  uint64_t p_full[2];     // [P buffer]: both column halves have written P
-  uint64_t pv_done[2];    // per P buffer: both PV MMAs that read it have finished
+  uint64_t s_full[2];     // [S buffer]: S of the buffer's tile is in TMEM
+  uint64_t p_full[2];     // [S buffer]: both column halves have written P over S
+  uint64_t pv_done[2];    // [S buffer]: both PV MMAs that read its P have finished
   uint64_t o_full, o_free;
   uint64_t item_full[2], item_empty[2];
   uint64_t xstate;        // softmax-state exchange between the halves at the end of an item
   uint64_t xread;         // both halves have read the exchanged state
   uint64_t teardown;
   int item_slot[2];
+  int item_T[2];          // tiles of the item in each slot
+  TileDesc desc[KVST];    // per ring stage, written before the stage's loads are armed
+  alignas(16) float qrow[128];  // producer: Q-bar_i of the item it routes (read as float4)
   uint32_t tmem_base;
   int abort_flag;
   float xm[2][BM];        // [column half][row] running max (log2 units)
@@ -123,24 +148,37 @@ struct Bars {
 static_assert(sizeof(Bars<Cfg<64>::KVST>) <= BAR_AREA && sizeof(Bars<Cfg<128>::KVST>) <= BAR_AREA,
               "barrier area");
 static_assert(QST == 1, "one Q buffer");
+static_assert(offsetof(Bars<3>, qrow) % 16 == 0 && offsetof(Bars<6>, qrow) % 16 == 0, "float4 access to qrow");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
 // unselected block, then the selected blocks in increasing order (one per
-// tile, or two with 64-token key blocks).
+// tile, or two with 64-token key blocks).  The selection words come from the
+// router's mask row in global memory, or (m == nullptr) from registers of the
+// warp: lane (w % 32) holds word w in rb0 (w < 32) or rb1.  Every lane of the
+// warp runs the same calls.
 struct TileIter {
   const uint32_t* m;
+  uint32_t rb0, rb1;
   int W, N, nchunk, pair;
   int chunk;     // next chunk to test
   int word;      // current mask word in the exact phase
   uint32_t bits; // remaining set bits of that word
   __device__ void init(const uint32_t* mrow, int W_, int N_, int nchunk_, int pair_) {
-    m = mrow; W = W_; N = N_; nchunk = nchunk_; pair = pair_;
+    m = mrow; rb0 = rb1 = 0; W = W_; N = N_; nchunk = nchunk_; pair = pair_;
     chunk = 0; word = -1; bits = 0;
+  }
+  __device__ __forceinline__ uint32_t load_word(int w) const {
+    if (m) return m[w];
+    return __shfl_sync(0xffffffffu, w < 32 ? rb0 : rb1, w & 31);
+  }
+  // unselected, in-range blocks of mask word w
+  __device__ __forceinline__ uint32_t unselected(int w) const {
+    return w < W ? (~load_word(w)) & valid_bits(w) : 0u;
   }
   __device__ __forceinline__ int next_selected() {
     while (bits == 0) {
       if (++word >= W) return -1;
-      bits = m[word];
+      bits = load_word(word);
     }
     const int b = __ffs(bits) - 1;
     bits &= bits - 1;
@@ -158,10 +196,7 @@ struct TileIter {
       const int c = chunk++;
       uint32_t un = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int w = c * 4 + q;
-        if (w < W) un |= (~m[w]) & valid_bits(w);
-      }
+      for (int q = 0; q < 4; ++q) un |= unselected(c * 4 + q);
       if (un) { kind = 0; idx = c; return true; }
     }
     idx = next_selected();
@@ -171,6 +206,67 @@ struct TileIter {
     return true;
   }
 };
+
+// Eq. 4 decided inside the kernel for query block `item`: the whole warp
+// forms s_ij = (Q-bar_i . K-bar_j) / sqrt(d) for every key block j, four
+// pooled keys per lane at a time, with the router's arithmetic (fp32, one
+// fused multiply-add per channel in channel order, then the scale), and keeps
+// the bits j with s_ij > tau_i as mask words in registers (W <= 64).  Returns
+// the item's tile count: pooled chunks holding an unselected block (with the
+// correction) plus the exact tiles.
+template <int HD>
+__device__ int route_row(const Params& p, int item, float* qrow, int lane, TileIter& ti) {
+  const int bh = item / p.Nq;
+  const float* qsrc = p.qbar + (size_t)item * HD;
+  for (int c = lane * 4; c < HD; c += 128)
+    *reinterpret_cast<float4*>(qrow + c) = __ldg(reinterpret_cast<const float4*>(qsrc + c));
+  __syncwarp();
+  const float tau = __ldg(p.tau + item);
+  const float* kb = p.kbar + (size_t)bh * p.Nk * HD;
+  ti.init(nullptr, p.W, p.Nk, p.chunks, p.pair);
+  int cnt = 0, used = 0;
+  const int nch = (p.Nk + 127) >> 7;
+  for (int c = 0; c < nch; ++c) {
+    float acc[4];
+    const float* kr[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = c * 128 + r * 32 + lane;
+      kr[r] = kb + (size_t)(j < p.Nk ? j : 0) * HD;  // rows past Nk read row 0 and are masked below
+      acc[r] = 0.f;
+    }
+#pragma unroll 4
+    for (int cc = 0; cc < HD; cc += 4) {
+      const float4 q4 = *reinterpret_cast<const float4*>(qrow + cc);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 k4 = __ldg(reinterpret_cast<const float4*>(kr[r] + cc));
+        acc[r] = fmaf(q4.x, k4.x, acc[r]);
+        acc[r] = fmaf(q4.y, k4.y, acc[r]);
+        acc[r] = fmaf(q4.z, k4.z, acc[r]);
+        acc[r] = fmaf(q4.w, k4.w, acc[r]);
+      }
+    }
+    bool any_unselected = false;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int w = c * 4 + r;  // keys 32w .. 32w + 31
+      const bool bit = (32 * w + lane < p.Nk) && (acc[r] * p.scale > tau);
+      const uint32_t word = __ballot_sync(0xffffffffu, bit);
+      if (w < p.W) {
+        if (lane == (w & 31)) {
+          if (w < 32) ti.rb0 = word;
+          else ti.rb1 = word;
+        }
+        cnt += __popc(word);
+        any_unselected |= ((~word) & ti.valid_bits(w)) != 0u;
+      }
+    }
+    used += any_unselected ? 1 : 0;
+  }
+  __syncwarp();  // qrow is rewritten for the next item
+  return (p.chunks ? used : 0) + (p.pair ? (cnt + 1) >> 1 : cnt);
+}
 
 // All 32 lanes wait; the outcome is made warp-uniform so that warp-wide
 // instructions that follow are never reached by part of a warp.
@@ -236,8 +332,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < QST; ++s) { mbar_init(&bars.q_full[s], 1); mbar_init(&bars.q_empty[s], 1); }
     for (int s = 0; s < KVST; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_free, SOFTMAX_WARPS);
+    mbar_init(&bars.s_full[0], 1);
+    mbar_init(&bars.s_full[1], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.p_full[s], SOFTMAX_WARPS);
       mbar_init(&bars.pv_done[s], 1);
@@ -282,13 +378,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) idx = atomicAdd(p.work_counter, 1);
       idx = __shfl_sync(0xffffffffu, idx, 0);
       const int item = idx < p.nitems ? p.order[idx] : -1;
+      TileIter ti;
+      int T = 0;
+      if (item >= 0) {
+        if (p.route_inkernel) {
+          T = route_row<HD>(p, item, bars.qrow, lane, ti);
+        } else {
+          ti.init(p.mask + (size_t)item * p.W, p.W, p.Nk, p.chunks, p.pair);
+          T = p.tiles[item];
+        }
+      }
       if (lane == 0) {
         bars.item_slot[slot] = item;
+        bars.item_T[slot] = T;
         mbar_arrive(&bars.item_full[slot]);
       }
       if (item < 0) break;
       const int bh = item / p.Nq, qi = item % p.Nq;
-      const int T = p.tiles[item];
       if (T == 0) continue;
       // Q tile into buffer q_uses % QST, once the item that used it last has
       // issued all its S MMAs
@@ -303,11 +409,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_3d(qdst + hd * SLAB, &tmQ, &bars.q_full[qb], hd * 64, qi * BM, bh, pol_q);
       }
       ++q_uses;
-      TileIter ti;
-      ti.init(p.mask + (size_t)item * p.W, p.W, p.Nk, p.chunks, p.pair);
       for (int n = 0; n < T; ++n) {
         int kind = 0, tidx = 0, tidx2 = -1;
         ti.next(kind, tidx, tidx2);
+        uint32_t vm[4] = {0u, 0u, 0u, 0u};
+        if (kind == 0) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) vm[q] = ti.unselected(tidx * 4 + q);
+        }
         const uint32_t gk = g + n;
         const int ks = gk % KVST;
         const int ku = gk / KVST;
@@ -316,6 +425,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (leader) {
           uint8_t* dk = smem + C::OFF_KV + (2 * ks) * TILE_BYTES;
           uint8_t* dv = dk + TILE_BYTES;
+          TileDesc& td = bars.desc[ks];  // published by the arrive below (release)
+          td.kind = kind;
+          td.idx = tidx;
+          td.idx2 = tidx2;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) td.vm[q] = vm[q];
           mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
           if (kind == 1 && p.pair) {
             // rows [0, 64) <- key block tidx, rows [64, 128) <- key block tidx2;
@@ -363,21 +478,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int item_local = 0;  // items with T > 0 processed
     bool issued = false;
     bool ok = true;
-    // S_gs = Q K_gs^T into the single S buffer, once the softmax has read S_{gs-1}
-    auto issue_s = [&](uint32_t gs, uint32_t sQ) -> bool {
+    // S_gs = Q K_gs^T into S buffer gs % 2.  The buffer last held tile gs - 2:
+    // the softmax read that S before handing over its P, and the PV that read
+    // the P was issued before this MMA by this thread, so it is done first.
+    // last: this is the item's last S; the Q buffer is released after it.
+    auto issue_s = [&](uint32_t gs, uint32_t sQ, bool last, int qb) -> bool {
       const int ks = gs % KVST;
       if (!wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 15)) return false;
-      if (gs >= 1 && !wait_warp(&bars.s_free, (gs - 1) & 1, bars, lim, 16)) return false;
       tc_fence_after();
       const uint32_t kbase = sKV + (2 * ks) * TILE_BYTES;
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * SLAB + (kk & 3) * 32;
-          mma_ss(tmem + TM_S, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                 IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + TM_S + (gs & 1) * 128, smem_desc_sw128(sQ + off, 16, 1024),
+                 smem_desc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars.s_full);
+        tc_commit(&bars.s_full[gs & 1]);
+        if (last) tc_commit(&bars.q_empty[qb]);  // every S MMA of this item has been issued
       }
       __syncwarp();
       return true;
@@ -395,7 +513,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + TM_O + h * 128, tmem + TM_P + pb * 64 + h * 32 + kk * 8,
+            mma_ts(tmem + TM_O + h * 128, tmem + TM_S + pb * 128 + h * 64 + kk * 8,
                    smem_desc_sw128(vbase + h * 8192 + kk * 2048, SLAB, 1024), IDESC_PV,
                    (first && kk == 0) ? 0u : 1u);
         }
@@ -409,24 +527,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int slot = it & 1;
       if (!(ok = wait_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 10))) break;
       const int item = bars.item_slot[slot];
+      const int T = bars.item_T[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (item < 0) break;
-      const int T = p.tiles[item];
       if (T == 0) continue;
       const int qb = item_local % QST;
       if (!(ok = wait_warp(&bars.q_full[qb], (item_local / QST) & 1, bars, lim, 11))) break;
       const uint32_t sQ = smem_u32(smem + C::OFF_Q + qb * TILE_BYTES);
-      // order: S_0, then for each tile n: S_{n+1}, PV_n
-      if (!(ok = issue_s(g, sQ))) break;
+      // order: S_0, S_1, then for each tile n: PV_n, S_{n+2}
+      if (!(ok = issue_s(g, sQ, T == 1, qb))) break;
       issued = true;
+      if (T > 1 && !(ok = issue_s(g + 1, sQ, T == 2, qb))) break;
       for (int n = 0; n < T && ok; ++n) {
-        if (n + 1 < T) {
-          if (!(ok = issue_s(g + n + 1, sQ))) break;
-        } else if (leader) {
-          tc_commit(&bars.q_empty[qb]);  // every S MMA of this item has been issued
-        }
         if (!(ok = issue_pv(g + n, n == 0))) break;
+        if (n + 2 < T && !(ok = issue_s(g + n + 2, sQ, n + 3 == T, qb))) break;
       }
       if (!ok) break;
       if (leader) tc_commit(&bars.o_full);
@@ -458,11 +573,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int slot = it & 1;
       if (!(ok = wait_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 20))) break;
       const int item = bars.item_slot[slot];
+      const int T = bars.item_T[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (item < 0) break;
       const int bh = item / p.Nq, qi = item % p.Nq;
-      const int T = p.tiles[item];
       const int n_rows = min(BM, p.L - qi * BM);
       __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD + ocol0;
       if (T == 0) {
@@ -470,21 +585,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int c = 0; c < HD / 2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
-      TileIter ti;
-      ti.init(p.mask + (size_t)item * p.W, p.W, p.Nk, p.chunks, p.pair);
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < T; ++n) {
-        int kind = 0, tidx = 0, tidx2 = -1;
-        ti.next(kind, tidx, tidx2);
         const uint32_t gs = g + n;
         const int pb = gs & 1;
-        if (!(ok = wait_warp(&bars.s_full, gs & 1, bars, lim, 21))) break;
+        const int ks = gs % KVST;
+        if (!(ok = wait_warp(&bars.s_full[pb], (gs >> 1) & 1, bars, lim, 21))) break;
+        // the tile's descriptor: S_gs being ready implies its stage was filled,
+        // and this (already complete) wait orders the producer's writes before
+        // the reads; the stage cannot refill before this warp hands over P
+        if (!(ok = wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 22))) break;
+        const int kind = bars.desc[ks].kind, tidx = bars.desc[ks].idx, tidx2 = bars.desc[ks].idx2;
         tc_fence_after();
         float x[64];
         {
           uint32_t r0[32], r1[32];
-          tmem_ld32(tmem + lane_off + TM_S + col0, r0);
-          tmem_ld32(tmem + lane_off + TM_S + col0 + 32, r1);
+          tmem_ld32(tmem + lane_off + TM_S + pb * 128 + col0, r0);
+          tmem_ld32(tmem + lane_off + TM_S + pb * 128 + col0 + 32, r1);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -492,9 +609,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             x[32 + c] = __uint_as_float(r1[c]);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.s_free);
 
         // valid key columns of this half of an exact tile: all 64 except in
         // the last (partial) key block and in a pair tile's empty second half
@@ -528,10 +642,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           } else {  // pooled chunk: unselected, in-range blocks only
             bias = p.bias_full;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int w = tidx * 4 + half * 2 + q;
-              vm[q] = (w < p.W) ? ((~p.mask[(size_t)item * p.W + w]) & ti.valid_bits(w)) : 0u;
-            }
+            for (int q = 0; q < 2; ++q) vm[q] = bars.desc[ks].vm[half * 2 + q];
             const int jl = p.Nk - 1 - tidx * BN - col0;
             if (jl >= 0 && jl < 64 && p.bias_last != p.bias_full) {
               sc = jl;
@@ -577,10 +688,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         const float2 s2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
         l += s2.x + s2.y;
-        // P buffer pb was last read by the PV of tile gs - 2; no wait is needed:
-        // the MMA thread issued that PV before S of tile gs, and the s_full
-        // commit it made after S fires only when all its earlier MMAs are done
-        tmem_st32(tmem + lane_off + TM_P + pb * 64 + half * 32, pk);
+        // P over the first 32 columns of this half's S (already in registers).
+        // The PV of tile gs - 2 read the previous P of this buffer; it was
+        // issued before S of tile gs, and the s_full commit made after that S
+        // fires only when all earlier MMAs are done, so no wait is needed
+        tmem_st32(tmem + lane_off + TM_S + pb * 128 + col0, pk);
         if (n > 0 && __any_sync(0xffffffffu, need)) {
           // O_h must hold every PV up to tile gs - 1 before it is rescaled
           const uint32_t gp = gs - 1;
@@ -715,7 +827,8 @@ cudaError_t launch_hd(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtens
 }  // namespace
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
-                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction) {
+                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction,
+                           int route_inkernel) {
   CUtensorMap mQ, mK, mV, mKb, mVb;
   // built for d in {64, 128}, query blocks of 128 tokens, key blocks of 128 or 64
   if (g.Bq != BM || (g.Bk != BN && g.Bk != BN / 2) || (g.d != 64 && g.d != 128)) return cudaErrorInvalidValue;
@@ -734,6 +847,10 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.out = static_cast<__nv_bfloat16*>(out);
   p.wait_limit_ns = wait_limit_ns;
   p.chunks = correction ? g.nchunk : 0;
+  p.route_inkernel = route_inkernel;
+  p.scale = 1.0f / sqrtf((float)g.d);  // the router's expression, evaluated the same way
+  p.qbar = s.qbar; p.kbar = s.kbar; p.tau = s.tau;
+  if (route_inkernel && (g.W > kInKernelMaxW || !s.tau)) return cudaErrorInvalidValue;
   if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
   return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
 }

@@ -34,7 +34,8 @@ struct Scratch {
   void* kbar_op;   // [bH, Nk, d]  mean key per block in the attention kernel's operand type
   void* vbar_op;   // [bH, Nk, d]  V-hat_j / n_j in the attention kernel's operand type
   float* kvar;     // [bH, d]      Var_j(K-bar_j,c), population (diagonal sigma only)
-  uint32_t* mask;  // [bH, Nq, W]  bit j of row i: key block j selected for query block i
+  uint32_t* mask;  // [bH, Nq, W]  bit j of row i: key block j selected for query block i (may be null)
+  float* tau;      // [bH, Nq]     tau_i of Eq. 4
   int32_t* counts; // [bH, Nq]     |S_i|
   int32_t* tiles;  // [bH, Nq]     tiles of the attention loop: |S_i| + pooled-key chunks used
   int32_t* order;  // [bH * Nq]    work items, head-major, heaviest first within a head
@@ -60,8 +61,12 @@ cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st);
 
 // Attention launches.
 // correction = 0: keep-or-drop (pooled-key tiles skipped, empty rows give 0).
+// route_inkernel != 0: the tensor-core kernel decides S_i itself from s.qbar,
+// s.kbar and s.tau (needs W <= 64) and never reads s.mask.
+constexpr int kInKernelMaxW = 64;
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
-                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction);
+                           const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction,
+                           int route_inkernel);
 cudaError_t launch_attn_simt(int dtype, const void* q, const void* k, const void* v, void* out,
                              const Geometry& g, const Scratch& s, cudaStream_t st, int correction);
 cudaError_t read_device_status(cudaStream_t st, int32_t* word);

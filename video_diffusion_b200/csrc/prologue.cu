@@ -158,7 +158,7 @@ constexpr int kRouteKC = 32;  // pooled keys staged in shared memory at a time
 // products over one key row.  Row pass: warp w takes query blocks w, w + 8, ...
 // kvar == nullptr: sigma_i from the row (Eq. 5); else the diagonal estimator.
 // tiles[i] counts the attention kernel's tiles: pooled-key chunks used plus the
-// selected blocks, two to a tile when pair != 0.
+// selected blocks, two to a tile when pair != 0.  mask and tau_out may be null.
 template <int D, int QPW>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __restrict__ qbar,
                                                               const float* __restrict__ kbar,
@@ -167,7 +167,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
                                                               int beta_mode, int correction, int pair,
                                                               uint32_t* __restrict__ mask,
                                                               int32_t* __restrict__ counts,
-                                                              int32_t* __restrict__ tiles) {
+                                                              int32_t* __restrict__ tiles,
+                                                              float* __restrict__ tau_out) {
   constexpr int QB = 8 * QPW;
   extern __shared__ float sm[];
   float* qs = sm;                          // [QB][D]
@@ -238,14 +239,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     else tau = fmaf(beta, sigma, mu);
 
     const size_t item = (size_t)bh * Nq + i0 + qi;
-    uint32_t* mrow = mask + item * W;
     int cnt = 0;
     for (int w = lane; w < W; w += 32) {
       uint32_t bits = 0;
       const int jb = w * 32;
       const int nb = min(32, Nk - jb);
       for (int b = 0; b < nb; ++b) bits |= (s[jb + b] > tau ? 1u : 0u) << b;
-      mrow[w] = bits;
+      if (mask) mask[item * W + w] = bits;
       cnt += __popc(bits);
     }
 #pragma unroll
@@ -275,6 +275,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     if (lane == 0) {
       counts[item] = cnt;
       tiles[item] = (pair ? (cnt + 1) >> 1 : cnt) + used;
+      if (tau_out) tau_out[item] = tau;
     }
   }
 }
@@ -364,7 +365,7 @@ static cudaError_t route_launch(const Geometry& g, const Scratch& s, float beta,
   dim3 grid((g.Nq + QB - 1) / QB, g.bH);
   route_kernel<D, QPW><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, g.W, g.nchunk,
                                                           1.0f / sqrtf((float)D), beta, beta_mode, correction,
-                                                          pair, s.mask, s.counts, s.tiles);
+                                                          pair, s.mask, s.counts, s.tiles, s.tau);
   return cudaGetLastError();
 }
 
