@@ -58,27 +58,22 @@ constexpr int QST = 1;  // Q buffers
 constexpr int NTHREADS = 320;
 constexpr int SOFTMAX_WARPS = 8;
 constexpr uint32_t SLAB = BM * 128;  // 16 KB: 64 bf16 columns of a 128-row tile, 128-byte swizzled
+constexpr uint32_t BAR_AREA = 3072;
+
 // Shared-memory plan for head dimension HD (64 or 128).  A Q, K or V tile is
-// HD / 64 slabs.  K and V have rings of their own: K is needed when S of a
-// tile is computed, V a tile later for PV, so the K ring is twice as deep and
-// its loads run further ahead (4 K and 2 V stages at d = 128, 8 and 4 at
-// d = 64).  Both stages of a tile are released together when its PV is done.
-// There is no room for alignment slack: the kernel checks that dynamic
-// shared memory starts on a 1024-byte boundary (the 128-byte swizzle needs
-// it) and reports an error instead of running if it does not.
+// HD / 64 slabs; the K+V ring gets as many stages as fit (3 at d = 128, 6 at
+// d = 64).  There is no room for alignment slack: the kernel checks that
+// dynamic shared memory starts on a 1024-byte boundary (the 128-byte swizzle
+// needs it) and reports an error instead of running if it does not.
 template <int HD>
 struct Cfg {
   static_assert(HD == 64 || HD == 128, "head dimension");
   static constexpr int NSLAB = HD / 64;
   static constexpr uint32_t TILE_BYTES = NSLAB * SLAB;
-  static constexpr int KST = HD == 128 ? 4 : 8;  // K stages
-  static constexpr int VST = KST / 2;            // V stages
-  static constexpr int LAG = KST - VST;          // V of tile t is loaded with K of tile t + LAG
+  static constexpr int KVST = HD == 128 ? 3 : 6;  // K+V stages
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + QST * TILE_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + KST * TILE_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + VST * TILE_BYTES;
-  static constexpr uint32_t BAR_AREA = HD == 128 ? 3072 : 4096;
+  static constexpr uint32_t OFF_KV = OFF_Q + QST * TILE_BYTES;  // stage s: K at +2s tiles, V at +2s+1
+  static constexpr uint32_t OFF_BAR = OFF_KV + 2 * KVST * TILE_BYTES;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA;
   static constexpr int OCHUNK = HD / 64;  // 32-column output chunks per softmax half
 };
@@ -136,14 +131,12 @@ struct TileDesc {
   uint32_t vm[4];
 };
 
-template <int KST, int VST>
+template <int KVST>
 struct Bars {
   uint64_t q_full[QST], q_empty[QST];
-  uint64_t k_full[KST], v_full[VST];
-  uint64_t stage_free[KST];  // [K stage]: the PV of its tile is done (frees the tile's K and V stages)
+  uint64_t kv_full[KVST], kv_empty[KVST];
   uint64_t s_full[2];     // [S buffer]: S of the buffer's tile is in TMEM
   uint64_t p_full[2];     // [S buffer]: both column halves have written P over S
-  uint64_t pv_done[2];    // [S buffer]: both PV MMAs that read its P have finished
   uint64_t o_full, o_free;
   uint64_t item_full[2], item_empty[2];
   uint64_t xstate;        // softmax-state exchange between the halves at the end of an item
@@ -151,18 +144,17 @@ struct Bars {
   uint64_t teardown;
   int item_slot[2];
   int item_T[2];          // tiles of the item in each slot
-  TileDesc desc[KST];     // per K stage, written before the stage's load is armed
+  TileDesc desc[KVST];    // per ring stage, written before the stage's loads are armed
   alignas(16) float qrow[128];  // producer: Q-bar_i of the item it routes (read as float4)
   uint32_t tmem_base;
   int abort_flag;
   float xm[2][BM];        // [column half][row] running max (log2 units)
   float xl[2][BM];        // [column half][row] row sum
 };
-template <int HD>
-using BarsOf = Bars<Cfg<HD>::KST, Cfg<HD>::VST>;
-static_assert(sizeof(BarsOf<64>) <= Cfg<64>::BAR_AREA && sizeof(BarsOf<128>) <= Cfg<128>::BAR_AREA, "barrier area");
+static_assert(sizeof(Bars<Cfg<64>::KVST>) <= BAR_AREA && sizeof(Bars<Cfg<128>::KVST>) <= BAR_AREA,
+              "barrier area");
 static_assert(QST == 1, "one Q buffer");
-static_assert(offsetof(BarsOf<64>, qrow) % 16 == 0 && offsetof(BarsOf<128>, qrow) % 16 == 0, "float4 access to qrow");
+static_assert(offsetof(Bars<3>, qrow) % 16 == 0 && offsetof(Bars<6>, qrow) % 16 == 0, "float4 access to qrow");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
 // unselected block, then the selected blocks in increasing order (one per
@@ -353,7 +345,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                    const __grid_constant__ CUtensorMap tmVb, const Params p) {
   using C = Cfg<HD>;
-  constexpr int KST = C::KST, VST = C::VST, LAG = C::LAG;
+  constexpr int KVST = C::KVST;
   constexpr int NSLAB = C::NSLAB;
   constexpr uint32_t TILE_BYTES = C::TILE_BYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -362,19 +354,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     return;
   }
   uint8_t* smem = smem_raw;
-  BarsOf<HD>& bars = *reinterpret_cast<BarsOf<HD>*>(smem + C::OFF_BAR);
+  Bars<KVST>& bars = *reinterpret_cast<Bars<KVST>*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < QST; ++s) { mbar_init(&bars.q_full[s], 1); mbar_init(&bars.q_empty[s], 1); }
-    for (int s = 0; s < KST; ++s) { mbar_init(&bars.k_full[s], 1); mbar_init(&bars.stage_free[s], 1); }
-    for (int s = 0; s < VST; ++s) mbar_init(&bars.v_full[s], 1);
+    for (int s = 0; s < KVST; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
     mbar_init(&bars.s_full[0], 1);
     mbar_init(&bars.s_full[1], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.p_full[s], SOFTMAX_WARPS);
-      mbar_init(&bars.pv_done[s], 1);
       mbar_init(&bars.item_full[s], 1);
       mbar_init(&bars.item_empty[s], 1 + SOFTMAX_WARPS);
     }
@@ -405,56 +395,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
     uint32_t g = 0;          // global tile counter
-    // tiles whose K / V loads were issued and Q tiles loaded (to let them land
-    // if the CTA abandons its work)
-    int nk_issued = 0, nv_issued = 0, q_uses = 0;
-    // V loads trail K loads by LAG tiles; lane (t % LAG) keeps what tile t's V
-    // load needs until then
-    int pend_kind = 0, pend_idx = 0, pend_idx2 = -1, pend_bh = 0;
+    // last K / V tile and number of Q tiles whose loads were issued (to let
+    // them land if the CTA abandons its work)
+    int gk_last = -1, q_uses = 0;
     bool ok = true;
-    // The stages of tile t + LAG - KST are free once its PV is done: then K of
-    // tile t + LAG and V of tile t may load.
-    auto wait_free = [&](int t_k) -> bool {
-      if (t_k < KST) return true;
-      return wait_warp(&bars.stage_free[t_k % KST], ((t_k / KST) - 1) & 1, bars, lim, 3);
-    };
-    auto load_v = [&](int tv) {
-      const int src = tv % LAG;
-      const int kind = __shfl_sync(0xffffffffu, pend_kind, src);
-      const int tidx = __shfl_sync(0xffffffffu, pend_idx, src);
-      const int tidx2 = __shfl_sync(0xffffffffu, pend_idx2, src);
-      const int vbh = __shfl_sync(0xffffffffu, pend_bh, src);
-      const int vs = tv % VST;
-      if (leader) {
-        uint8_t* dv = smem + C::OFF_V + vs * TILE_BYTES;
-        mbar_arrive_expect_tx(&bars.v_full[vs], TILE_BYTES);
-        if (kind == 1 && p.pair) {
-          const int j2 = tidx2 >= 0 ? tidx2 : tidx;
-#pragma unroll
-          for (int hd = 0; hd < NSLAB; ++hd) {
-            tma_load_3d(dv + hd * SLAB, &tmV, &bars.v_full[vs], hd * 64, tidx * 64, vbh, pol_kv);
-            tma_load_3d(dv + hd * SLAB + 64 * 128, &tmV, &bars.v_full[vs], hd * 64, j2 * 64, vbh, pol_kv);
-          }
-        } else {
-          const CUtensorMap* mv = kind ? &tmV : &tmVb;
-#pragma unroll
-          for (int hd = 0; hd < NSLAB; ++hd)
-            tma_load_3d(dv + hd * SLAB, mv, &bars.v_full[vs], hd * 64, tidx * BN, vbh, pol_kv);
-        }
-      }
-      nv_issued = tv + 1;
-    };
     for (int it = 0;; ++it) {
       const int slot = it & 1;
-      // The V loads still trailing the previous item's K loads go out first:
-      // the MMA thread needs them to finish that item, and both waits below
-      // (an item slot, the Q buffer) may depend on it having done so.  Their
-      // stages free up as the PVs issued before them finish.
-      for (int tv = nv_issued; ok && tv < nk_issued; ++tv) {
-        if (!(ok = wait_free(tv + LAG))) break;
-        load_v(tv);
-      }
-      if (!ok) break;
       if (it >= 2 && !(ok = wait_warp(&bars.item_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 1))) break;
       int idx = 0;
       if (lane == 0) idx = atomicAdd(p.work_counter, 1);
@@ -499,58 +445,54 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) vm[q] = ti.unselected(tidx * 4 + q);
         }
-        const int gk = (int)g + n;
-        const int ks = gk % KST;
-        if (!(ok = wait_free(gk))) break;
-        if (gk - LAG >= nv_issued) load_v(gk - LAG);  // V of the item's earlier tiles
-        if (lane == gk % LAG) {
-          pend_kind = kind;
-          pend_idx = tidx;
-          pend_idx2 = tidx2;
-          pend_bh = bh;
-        }
+        const uint32_t gk = g + n;
+        const int ks = gk % KVST;
+        const int ku = gk / KVST;
+        // stage ks is free once the PV of its previous tile has finished
+        if (ku > 0 && !(ok = wait_warp(&bars.kv_empty[ks], (ku - 1) & 1, bars, lim, 3))) break;
         if (leader) {
-          uint8_t* dk = smem + C::OFF_K + ks * TILE_BYTES;
+          uint8_t* dk = smem + C::OFF_KV + (2 * ks) * TILE_BYTES;
+          uint8_t* dv = dk + TILE_BYTES;
           TileDesc& td = bars.desc[ks];  // published by the arrive below (release)
           td.kind = kind;
           td.idx = tidx;
           td.idx2 = tidx2;
 #pragma unroll
           for (int q = 0; q < 4; ++q) td.vm[q] = vm[q];
-          mbar_arrive_expect_tx(&bars.k_full[ks], TILE_BYTES);
+          mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
           if (kind == 1 && p.pair) {
             // rows [0, 64) <- key block tidx, rows [64, 128) <- key block tidx2;
             // a tile with one block repeats it in the second half (masked out)
             const int j2 = tidx2 >= 0 ? tidx2 : tidx;
 #pragma unroll
             for (int hd = 0; hd < NSLAB; ++hd) {
-              tma_load_3d(dk + hd * SLAB, &tmK, &bars.k_full[ks], hd * 64, tidx * 64, bh, pol_kv);
-              tma_load_3d(dk + hd * SLAB + 64 * 128, &tmK, &bars.k_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+              tma_load_3d(dk + hd * SLAB, &tmK, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+              tma_load_3d(dk + hd * SLAB + 64 * 128, &tmK, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+              tma_load_3d(dv + hd * SLAB, &tmV, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+              tma_load_3d(dv + hd * SLAB + 64 * 128, &tmV, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
             }
           } else {
             const CUtensorMap* mk = kind ? &tmK : &tmKb;
+            const CUtensorMap* mv = kind ? &tmV : &tmVb;
 #pragma unroll
-            for (int hd = 0; hd < NSLAB; ++hd)
-              tma_load_3d(dk + hd * SLAB, mk, &bars.k_full[ks], hd * 64, tidx * BN, bh, pol_kv);
+            for (int hd = 0; hd < NSLAB; ++hd) {
+              tma_load_3d(dk + hd * SLAB, mk, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
+              tma_load_3d(dv + hd * SLAB, mv, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
+            }
           }
         }
-        nk_issued = gk + 1;
+        gk_last = (int)gk;
       }
       if (!ok) break;
       g += T;
     }
-    // the V loads still trailing the last K loads
-    for (int tv = nv_issued; ok && !bars.abort_flag && tv < nk_issued; ++tv) {
-      if (!(ok = wait_free(tv + LAG))) break;
-      load_v(tv);
-    }
     if (!ok || bars.abort_flag) {
       // let every copy this warp started land before the CTA exits: the last
       // use of each ring stage is one of the ring's last issued tiles
-      for (int t = nk_issued - KST; t < nk_issued; ++t)
-        if (t >= 0) mbar_wait(&bars.k_full[t % KST], (t / KST) & 1, nullptr, &g_sol_status, 0, lim);
-      for (int t = nv_issued - VST; t < nv_issued; ++t)
-        if (t >= 0) mbar_wait(&bars.v_full[t % VST], (t / VST) & 1, nullptr, &g_sol_status, 0, lim);
+      for (int back = 0; back < KVST; ++back) {
+        const int gk = gk_last - back;
+        if (gk >= 0) mbar_wait(&bars.kv_full[gk % KVST], (gk / KVST) & 1, nullptr, &g_sol_status, 0, lim);
+      }
       if (q_uses > 0) mbar_wait(&bars.q_full[0], (q_uses - 1) & 1, nullptr, &g_sol_status, 0, lim);
     }
     __syncwarp();
@@ -559,7 +501,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const bool leader = elect_one();
     constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-    const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
+    // Shared-memory descriptors of the first ring stage and of the Q buffer;
+    // a stage or a K-step only moves the start address, the low 14-bit field
+    // (address / 16, no carry: shared memory is < 256 KB)
+    constexpr uint32_t TILE16 = TILE_BYTES >> 4;
+    const uint64_t dK0 = smem_desc_sw128(smem_u32(smem + C::OFF_KV), 16, 1024);
+    const uint64_t dV0 = smem_desc_sw128(smem_u32(smem + C::OFF_KV) + TILE_BYTES, SLAB, 1024);
+    const uint64_t dQ = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
+    static_assert(QST == 1, "one Q descriptor");
     uint32_t g = 0;
     int item_local = 0;  // items with T > 0 processed
     bool issued = false;
@@ -568,17 +517,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // the softmax read that S before handing over its P, and the PV that read
     // the P was issued before this MMA by this thread, so it is done first.
     // last: this is the item's last S; the Q buffer is released after it.
-    auto issue_s = [&](uint32_t gs, uint32_t sQ, bool last, int qb) -> bool {
-      const int ks = gs % KST;
-      if (!wait_warp(&bars.k_full[ks], (gs / KST) & 1, bars, lim, 15)) return false;
+    auto issue_s = [&](uint32_t gs, bool last, int qb) -> bool {
+      const int ks = gs % KVST;
+      if (!wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 15)) return false;
       tc_fence_after();
-      const uint32_t kbase = sK + ks * TILE_BYTES;
       if (leader) {
+        const uint64_t dK = dK0 + (uint64_t)(2 * ks * TILE16);
+        const uint32_t tS = tmem + TM_S + (gs & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * SLAB + (kk & 3) * 32;
-          mma_ss(tmem + TM_S + (gs & 1) * 128, smem_desc_sw128(sQ + off, 16, 1024),
-                 smem_desc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * SLAB + (kk & 3) * 32) >> 4;
+          mma_ss(tS, dQ + off, dK + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars.s_full[gs & 1]);
         if (last) tc_commit(&bars.q_empty[qb]);  // every S MMA of this item has been issued
@@ -589,23 +538,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // O_h += P_h V_h for both halves of tile gp (its V arrived with its K)
     auto issue_pv = [&](uint32_t gp, bool first) -> bool {
       const int pb = gp & 1;
-      const int vs = gp % VST;
+      const int ks = gp % KVST;
       if (first && item_local > 0 && !wait_warp(&bars.o_free, (item_local - 1) & 1, bars, lim, 14)) return false;
       if (!wait_warp(&bars.p_full[pb], (gp >> 1) & 1, bars, lim, 12)) return false;
-      if (!wait_warp(&bars.v_full[vs], (gp / VST) & 1, bars, lim, 13)) return false;
       tc_fence_after();
-      const uint32_t vbase = sV + vs * TILE_BYTES;
       if (leader) {
+        const uint64_t dV = dV0 + (uint64_t)(2 * ks * TILE16);
+        const uint32_t tP = tmem + TM_S + pb * 128;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + TM_O + h * 128, tmem + TM_S + pb * 128 + h * 64 + kk * 8,
-                   smem_desc_sw128(vbase + h * 8192 + kk * 2048, SLAB, 1024), IDESC_PV,
+            mma_ts(tmem + TM_O + h * 128, tP + h * 64 + kk * 8, dV + ((h * 8192 + kk * 2048) >> 4), IDESC_PV,
                    (first && kk == 0) ? 0u : 1u);
         }
-        tc_commit(&bars.stage_free[gp % KST]);
-        tc_commit(&bars.pv_done[pb]);
+        // frees the tile's stage and tells the softmax that O holds this PV
+        tc_commit(&bars.kv_empty[ks]);
       }
       __syncwarp();
       return true;
@@ -621,14 +569,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (T == 0) continue;
       const int qb = item_local % QST;
       if (!(ok = wait_warp(&bars.q_full[qb], (item_local / QST) & 1, bars, lim, 11))) break;
-      const uint32_t sQ = smem_u32(smem + C::OFF_Q + qb * TILE_BYTES);
       // order: S_0, S_1, then for each tile n: PV_n, S_{n+2}
-      if (!(ok = issue_s(g, sQ, T == 1, qb))) break;
+      if (!(ok = issue_s(g, T == 1, qb))) break;
       issued = true;
-      if (T > 1 && !(ok = issue_s(g + 1, sQ, T == 2, qb))) break;
+      if (T > 1 && !(ok = issue_s(g + 1, T == 2, qb))) break;
       for (int n = 0; n < T && ok; ++n) {
         if (!(ok = issue_pv(g + n, n == 0))) break;
-        if (n + 2 < T && !(ok = issue_s(g + n + 2, sQ, n + 3 == T, qb))) break;
+        if (n + 2 < T && !(ok = issue_s(g + n + 2, n + 3 == T, qb))) break;
       }
       if (!ok) break;
       if (leader) tc_commit(&bars.o_full);
@@ -676,12 +623,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int n = 0; n < T; ++n) {
         const uint32_t gs = g + n;
         const int pb = gs & 1;
-        const int ks = gs % KST;
+        const int ks = gs % KVST;
         if (!(ok = wait_warp(&bars.s_full[pb], (gs >> 1) & 1, bars, lim, 21))) break;
-        // the tile's descriptor: S_gs being ready implies its K stage was
-        // filled, and this (already complete) wait orders the producer's writes
-        // before the reads; the stage cannot refill before this tile's PV
-        if (!(ok = wait_warp(&bars.k_full[ks], (gs / KST) & 1, bars, lim, 22))) break;
+        // the tile's descriptor: S_gs being ready implies its stage was filled,
+        // and this (already complete) wait orders the producer's writes before
+        // the reads; the stage cannot refill before this warp hands over P
+        if (!(ok = wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 22))) break;
         const int kind = bars.desc[ks].kind, tidx = bars.desc[ks].idx, tidx2 = bars.desc[ks].idx2;
         tc_fence_after();
         float x[64];
@@ -767,7 +714,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (n > 0 && __any_sync(0xffffffffu, need)) {
           // O_h must hold every PV up to tile gs - 1 before it is rescaled
           const uint32_t gp = gs - 1;
-          if (!(ok = wait_warp(&bars.pv_done[gp & 1], (gp >> 1) & 1, bars, lim, 23))) break;
+          if (!(ok = wait_warp(&bars.kv_empty[gp % KVST], (gp / KVST) & 1, bars, lim, 23))) break;
           tc_fence_after();
 #pragma unroll
           for (int q = 0; q < HD / 32; ++q) {
