@@ -129,6 +129,15 @@ uint64_t wait_limit_ns() {
   return kDefaultWaitLimitNs;
 }
 
+// Failure-detection test hook: SOL_ATTN_TEST_STALL=1 makes the tensor-core
+// kernel's first wait in every CTA unsatisfiable, so that (with a short
+// SOL_ATTN_WAIT_LIMIT_NS) the bounded wait runs out and the kernel reports
+// SOL_ERR_DEVICE_TIMEOUT through sol_attn_device_status instead of hanging.
+int test_stall() {
+  const char* e = std::getenv("SOL_ATTN_TEST_STALL");
+  return (e && *e && *e != '0') ? 1 : 0;
+}
+
 int record(void* const* events, int i, cudaStream_t st) {
   if (!events || !events[i]) return SOL_OK;
   return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
@@ -171,7 +180,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   if (use_tc) {
     e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) goto done;
-    e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), correction, inkernel);
+    e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), correction, inkernel, test_stall());
   } else {
     e = sol::launch_attn_simt(in_dtype, q, k, v, out, g, s, st, correction);
   }

@@ -86,12 +86,13 @@ constexpr uint32_t TM_S = 0, TM_O = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 // A share of the probabilities goes through an FMA-pipe polynomial exp2
-// instead of the MUFU ex2 unit: NPOLY of every 8 column pairs.  Per tile and
-// scheduler the two softmax warps then need about 900 issue slots and keep
-// the MUFU unit (4 lanes per cycle) busy for about 770 cycles; 3 of 8 shifts
-// the balance the other way (measured on Wan 720p: 2 of 8 is the fastest of
-// 0 to 3, by a few per cent).
-constexpr int NPOLY = 2;
+// instead of the MUFU ex2 unit: NPOLY of every 8 column pairs.  The softmax
+// warps are bound by issue slots rather than by MUFU throughput (4 lanes per
+// cycle per scheduler), above all on the schedulers that also host the
+// producer and the MMA warp, and the polynomial costs five times the issue
+// slots of MUFU: measured on Wan 720p, 0 or 1 of 8 is fastest, 3 of 8 about
+// 3 % slower.
+constexpr int NPOLY = 1;
 template <int NP>
 __host__ __device__ constexpr bool poly_pair(int pair) {
   return NP >= 3   ? ((pair & 7) == 2 || (pair & 7) == 5 || (pair & 7) == 7)
@@ -117,6 +118,7 @@ struct Params {
   // S_i from the fp32 pooled vectors and the router's tau_i instead of reading
   // the mask; the arithmetic is the router's, so the sets are identical
   int route_inkernel;
+  int test_stall;       // failure-detection tests: the CTA's first S is never signalled
   float scale;          // 1/sqrt(d) as the router computes it
   const float* qbar;    // [bH, Nq, d] fp32
   const float* kbar;    // [bH, Nk, d] fp32
@@ -529,7 +531,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint32_t off = ((kk >> 2) * SLAB + (kk & 3) * 32) >> 4;
           mma_ss(tS, dQ + off, dK + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars.s_full[gs & 1]);
+        if (!(p.test_stall && gs == 0)) tc_commit(&bars.s_full[gs & 1]);
         if (last) tc_commit(&bars.q_empty[qb]);  // every S MMA of this item has been issued
       }
       __syncwarp();
@@ -846,7 +848,7 @@ cudaError_t launch_hd(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtens
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
                            const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction,
-                           int route_inkernel) {
+                           int route_inkernel, int test_stall) {
   CUtensorMap mQ, mK, mV, mKb, mVb;
   // built for d in {64, 128}, query blocks of 128 tokens, key blocks of 128 or 64
   if (g.Bq != BM || (g.Bk != BN && g.Bk != BN / 2) || (g.d != 64 && g.d != 128)) return cudaErrorInvalidValue;
@@ -866,6 +868,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.wait_limit_ns = wait_limit_ns;
   p.chunks = correction ? g.nchunk : 0;
   p.route_inkernel = route_inkernel;
+  p.test_stall = test_stall;
   p.scale = 1.0f / sqrtf((float)g.d);  // the router's expression, evaluated the same way
   p.qbar = s.qbar; p.kbar = s.kbar; p.tau = s.tau;
   if (route_inkernel && (g.W > kInKernelMaxW || !s.tau)) return cudaErrorInvalidValue;

@@ -64,9 +64,12 @@ cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st);
 // route_inkernel != 0: the tensor-core kernel decides S_i itself from s.qbar,
 // s.kbar and s.tau (needs W <= 64) and never reads s.mask.
 constexpr int kInKernelMaxW = 64;
+// test_stall != 0 (failure-detection tests only): the MMA thread of every CTA
+// never signals its first S, so the waits on it run out and the kernel takes
+// its abort path.
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
                            const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction,
-                           int route_inkernel);
+                           int route_inkernel, int test_stall = 0);
 cudaError_t launch_attn_simt(int dtype, const void* q, const void* k, const void* v, void* out,
                              const Geometry& g, const Scratch& s, cudaStream_t st, int correction);
 cudaError_t read_device_status(cudaStream_t st, int32_t* word);
