@@ -38,12 +38,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def kernel_source_digest() -> str:
-    """sha256 over the attention kernel's sources (the profile's counters are
-    only reported while the kernel is unchanged since they were taken)."""
+    """sha256 over the attention kernel's sources with comments and blank
+    lines removed (the profile's counters are only reported while the code is
+    unchanged since they were taken; editing a comment does not count)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in ("attn_tc.cu", "sm100.cuh", "common.cuh"):
-        h.update(open(os.path.join(ROOT, "video_diffusion_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "video_diffusion_b200", "csrc", f)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip()).encode())
     return h.hexdigest()
 
 
@@ -517,7 +522,9 @@ def main():
         "roofline": {"kernel": attention_kernel_name(wl, blk), "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": profiled_traffic(workload_key(wl, args)),
-                     "peak_source": f"{peaks['source']} bf16 burst"},
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": (achieved / float(peaks["bf16_tflops_sustained"])
+                                           if peaks.get("bf16_tflops_sustained") else None)},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": (5 if diag else 4) * args.steps,

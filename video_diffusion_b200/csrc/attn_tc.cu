@@ -1,11 +1,13 @@
 // attn_tc.cu -- the Sol-Attn attention loop on the 5th-generation tensor cores
-// (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, d = 128, query
-// blocks of 128 tokens, key blocks of 128 or 64 tokens.
+// (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, d = 128 or 64,
+// query blocks of 128 tokens, key blocks of 128 or 64 tokens.
 //
-// The MMA warp's barrier operations, not the tensor pipe, set the pace of
-// the key loop (each wait or commit costs a few hundred cycles while the
-// softmax warps keep the memory pipes busy), so the handoffs per tile are
-// kept to three waits and three commits.
+// What sets the pace is issue slots on the four schedulers, not the tensor
+// pipe: the softmax of a 128 x 128 tile takes about 900 issue slots per
+// scheduler, and the producer and MMA warps take theirs from the softmax
+// warps that share a scheduler with them.  So the control warps are kept
+// lean (descriptors built once, one commit per MMA group, waits that probe
+// before they block) and most exponentials go to the MUFU unit.
 //
 // One online-softmax pass per query block i (Sol-Attn visual explainer, "One
 // online-softmax state": exact and approximate terms share the running
