@@ -23,12 +23,14 @@
 //     128-column tile holds two selected blocks, one per softmax column half
 //     (an odd count leaves the last tile's second half masked out).
 //
-// Persistent CTAs, one per SM, 320 threads:
+// Persistent CTAs, one per SM, 352 threads:
 //   warp 0      TMA producer: fetches work items, loads the Q tile and each
 //               tile's K and V (or K-bar and V-bar) together into a 3-stage
 //               ring (a tile copy takes about a tile's worth of time when
 //               every SM loads at once, so copies run up to three tiles ahead)
 //   warp 1      TMEM owner and tcgen05.mma issuer (one elected lane)
+//   warp 10     in-kernel routing only: fetches the work items and decides
+//               each one's selection ahead of the producer
 //   warps 2..9  softmax, two column halves: half h owns the 64 keys
 //               [64h, 64h + 64) of every tile, one query row per thread (its
 //               warp's TMEM lane quadrant).  Each half keeps its own running
@@ -57,7 +59,8 @@ namespace {
 
 constexpr int BM = 128, BN = 128;
 constexpr int QST = 1;  // Q buffers
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 352;
+constexpr int ROUTER_WARP = 10;  // in-kernel routing: scores the items ahead of the producer
 constexpr int SOFTMAX_WARPS = 8;
 constexpr uint32_t SLAB = BM * 128;  // 16 KB: 64 bf16 columns of a 128-row tile, 128-byte swizzled
 constexpr uint32_t BAR_AREA = 3072;
@@ -149,7 +152,11 @@ struct Bars {
   int item_slot[2];
   int item_T[2];          // tiles of the item in each slot
   TileDesc desc[KVST];    // per ring stage, written before the stage's loads are armed
-  alignas(16) float qrow[128];  // producer: Q-bar_i of the item it routes (read as float4)
+  // in-kernel routing: the router warp hands each item (index, tile count,
+  // selection words) to the producer through two slots
+  uint64_t rq_full[2], rq_empty[2];
+  int rq_item[2], rq_T[2];
+  uint32_t rq_bits[2][64];
   uint32_t tmem_base;
   int abort_flag;
   float xm[2][BM];        // [column half][row] running max (log2 units)
@@ -158,7 +165,6 @@ struct Bars {
 static_assert(sizeof(Bars<Cfg<64>::KVST>) <= BAR_AREA && sizeof(Bars<Cfg<128>::KVST>) <= BAR_AREA,
               "barrier area");
 static_assert(QST == 1, "one Q buffer");
-static_assert(offsetof(Bars<3>, qrow) % 16 == 0 && offsetof(Bars<6>, qrow) % 16 == 0, "float4 access to qrow");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
 // unselected block, then the selected blocks in increasing order (one per
@@ -221,19 +227,19 @@ struct TileIter {
 // forms s_ij = (Q-bar_i . K-bar_j) / sqrt(d) for every key block j, four
 // pooled keys per lane at a time, with the router's arithmetic (fp32, one
 // fused multiply-add per channel in channel order, then the scale), and keeps
-// the bits j with s_ij > tau_i as mask words in registers (W <= 64).  Returns
-// the item's tile count: pooled chunks holding an unselected block (with the
-// correction) plus the exact tiles.
+// the bits j with s_ij > tau_i as mask words: lane (w % 32) gets word w in rb0
+// (w < 32) or rb1 (W <= 64).  Q-bar_i stays in registers (lane l holds
+// channels 4l .. 4l + 3) and is broadcast with shuffles.  Returns the item's
+// tile count: pooled chunks holding an unselected block (with the correction)
+// plus the exact tiles.
 template <int HD>
-__device__ int route_row(const Params& p, int item, float* qrow, int lane, TileIter& ti) {
+__device__ int route_row(const Params& p, int item, int lane, uint32_t& rb0, uint32_t& rb1) {
   const int bh = item / p.Nq;
-  const float* qsrc = p.qbar + (size_t)item * HD;
-  for (int c = lane * 4; c < HD; c += 128)
-    *reinterpret_cast<float4*>(qrow + c) = __ldg(reinterpret_cast<const float4*>(qsrc + c));
-  __syncwarp();
+  float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane * 4 < HD) qv = __ldg(reinterpret_cast<const float4*>(p.qbar + (size_t)item * HD) + lane);
   const float tau = __ldg(p.tau + item);
   const float* kb = p.kbar + (size_t)bh * p.Nk * HD;
-  ti.init(nullptr, p.W, p.Nk, p.chunks, p.pair);
+  rb0 = rb1 = 0u;
   int cnt = 0, used = 0;
   const int nch = (p.Nk + 127) >> 7;
   for (int c = 0; c < nch; ++c) {
@@ -247,14 +253,15 @@ __device__ int route_row(const Params& p, int item, float* qrow, int lane, TileI
     }
 #pragma unroll 4
     for (int cc = 0; cc < HD; cc += 4) {
-      const float4 q4 = *reinterpret_cast<const float4*>(qrow + cc);
+      const float qx = __shfl_sync(0xffffffffu, qv.x, cc >> 2), qy = __shfl_sync(0xffffffffu, qv.y, cc >> 2);
+      const float qz = __shfl_sync(0xffffffffu, qv.z, cc >> 2), qw = __shfl_sync(0xffffffffu, qv.w, cc >> 2);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const float4 k4 = __ldg(reinterpret_cast<const float4*>(kr[r] + cc));
-        acc[r] = fmaf(q4.x, k4.x, acc[r]);
-        acc[r] = fmaf(q4.y, k4.y, acc[r]);
-        acc[r] = fmaf(q4.z, k4.z, acc[r]);
-        acc[r] = fmaf(q4.w, k4.w, acc[r]);
+        acc[r] = fmaf(qx, k4.x, acc[r]);
+        acc[r] = fmaf(qy, k4.y, acc[r]);
+        acc[r] = fmaf(qz, k4.z, acc[r]);
+        acc[r] = fmaf(qw, k4.w, acc[r]);
       }
     }
     bool any_unselected = false;
@@ -265,16 +272,17 @@ __device__ int route_row(const Params& p, int item, float* qrow, int lane, TileI
       const uint32_t word = __ballot_sync(0xffffffffu, bit);
       if (w < p.W) {
         if (lane == (w & 31)) {
-          if (w < 32) ti.rb0 = word;
-          else ti.rb1 = word;
+          if (w < 32) rb0 = word;
+          else rb1 = word;
         }
         cnt += __popc(word);
-        any_unselected |= ((~word) & ti.valid_bits(w)) != 0u;
+        const int nb = p.Nk - w * 32;
+        const uint32_t valid = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+        any_unselected |= ((~word) & valid) != 0u;
       }
     }
     used += any_unselected ? 1 : 0;
   }
-  __syncwarp();  // qrow is rewritten for the next item
   return (p.chunks ? used : 0) + (p.pair ? (cnt + 1) >> 1 : cnt);
 }
 
@@ -377,6 +385,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars.o_full, 1);
     mbar_init(&bars.o_free, SOFTMAX_WARPS);
     mbar_init(&bars.teardown, 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars.rq_full[s], 1); mbar_init(&bars.rq_empty[s], 1); }
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -406,16 +415,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int it = 0;; ++it) {
       const int slot = it & 1;
       if (it >= 2 && !(ok = wait_warp(&bars.item_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 1))) break;
-      int idx = 0;
-      if (lane == 0) idx = atomicAdd(p.work_counter, 1);
-      idx = __shfl_sync(0xffffffffu, idx, 0);
-      const int item = idx < p.nitems ? p.order[idx] : -1;
+      int item = -1, T = 0;
       TileIter ti;
-      int T = 0;
-      if (item >= 0) {
-        if (p.route_inkernel) {
-          T = route_row<HD>(p, item, bars.qrow, lane, ti);
-        } else {
+      if (p.route_inkernel) {
+        // the router warp has fetched and scored the item already
+        if (!(ok = wait_warp(&bars.rq_full[slot], (it >> 1) & 1, bars, lim, 4))) break;
+        item = bars.rq_item[slot];
+        T = bars.rq_T[slot];
+        ti.init(bars.rq_bits[slot], p.W, p.Nk, p.chunks, p.pair);
+      } else {
+        int idx = 0;
+        if (lane == 0) idx = atomicAdd(p.work_counter, 1);
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        item = idx < p.nitems ? p.order[idx] : -1;
+        if (item >= 0) {
           ti.init(p.mask + (size_t)item * p.W, p.W, p.Nk, p.chunks, p.pair);
           T = p.tiles[item];
         }
@@ -427,7 +440,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (item < 0) break;
       const int bh = item / p.Nq, qi = item % p.Nq;
-      if (T == 0) continue;
+      // the router's slot is released once this item's selection words are no
+      // longer read (after its last tile is issued)
+      auto release_route_slot = [&]() {
+        if (p.route_inkernel && lane == 0) mbar_arrive(&bars.rq_empty[slot]);
+      };
+      if (T == 0) {
+        release_route_slot();
+        continue;
+      }
       // Q tile into buffer q_uses % QST, once the item that used it last has
       // issued all its S MMAs
       const int qb = q_uses % QST;
@@ -488,6 +509,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         gk_last = (int)gk;
       }
       if (!ok) break;
+      release_route_slot();
       g += T;
     }
     if (!ok || bars.abort_flag) {
@@ -594,6 +616,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait(&bars.teardown, 0, nullptr, &g_sol_status, 0, lim);
     }
     __syncwarp();
+  } else if (warp == ROUTER_WARP) {
+    // ================================================================ router (in-kernel routing only)
+    bool ok = true;
+    for (int it = 0; p.route_inkernel; ++it) {
+      const int slot = it & 1;
+      if (it >= 2 && !(ok = wait_warp(&bars.rq_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 5))) break;
+      int idx = 0;
+      if (lane == 0) idx = atomicAdd(p.work_counter, 1);
+      idx = __shfl_sync(0xffffffffu, idx, 0);
+      const int item = idx < p.nitems ? p.order[idx] : -1;
+      int T = 0;
+      if (item >= 0) {
+        uint32_t rb0, rb1;
+        T = route_row<HD>(p, item, lane, rb0, rb1);
+        if (lane < p.W) bars.rq_bits[slot][lane] = rb0;
+        if (32 + lane < p.W) bars.rq_bits[slot][32 + lane] = rb1;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        bars.rq_item[slot] = item;
+        bars.rq_T[slot] = T;
+        mbar_arrive(&bars.rq_full[slot]);
+      }
+      if (item < 0) break;
+    }
+    (void)ok;
   } else {
     // ================================================================ softmax + epilogue
     const int half = (warp - 2) >> 2;     // column half of every S tile this warp owns
