@@ -48,6 +48,27 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row(cuda_device):
     assert api.device_status() == 0
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("d,bk", [(128, 64), (64, 128)])
+def test_noalloc_other_shapes_match_forward(cuda_device, d, bk):
+    """64-token key blocks (two per tensor-core tile) and 64-wide heads take
+    the same kernels through the fixed scratch."""
+    f = _fn()
+    stream = torch.cuda.current_stream()
+    Q, K, V = I.make_qkv((5, 9, 40), heads=3, d=d, seed=23, device=cuda_device)  # L = 1800 (ragged)
+    ref = api.forward(Q, K, V, 1.04, (128, bk))
+    for _ in range(2):
+        out = torch.full_like(Q, float("nan"))
+        b, h, L, dd = Q.shape
+        rc = f(Q.data_ptr(), K.data_ptr(), V.data_ptr(), out.data_ptr(), b, h, L, dd, 128, bk, 1.04,
+               stream.cuda_stream)
+        assert rc == 0, api.status_string(rc)
+        torch.cuda.synchronize()
+        assert not torch.isnan(out).any()
+        P.check_close(out.double().cpu().numpy(), ref.double().cpu().numpy(), torch.bfloat16, "noalloc vs forward")
+    assert api.device_status() == 0
+
+
 def test_noalloc_rejects_calls_larger_than_its_scratch():
     f = _fn()
     fake = 0x10000  # never dereferenced: the size check comes before any CUDA call
