@@ -302,3 +302,18 @@ def test_route_in_kernel_with_keep_or_drop_and_diagonal_sigma():
         b = api.forward_ex(Q, K, V, 1.04, 128, route_in_kernel=True, **kw)
         torch.cuda.synchronize()
         assert torch.equal(a, b), kw
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_output_aligned_to_16_bytes_only(d):
+    """The kernel writes rows with 32-byte stores when the output allows it;
+    a 16-byte-aligned (not 32-byte-aligned) output takes the 16-byte stores
+    and gives the same bits."""
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=d, seed=24, device="cuda")
+    ref = api.forward(Q, K, V, 1.04, 128)
+    buf = torch.empty(Q.numel() + 8, dtype=Q.dtype, device="cuda")
+    out = buf[8:].view(Q.shape)  # 16 bytes past a 256-byte boundary
+    assert out.data_ptr() % 32 == 16
+    api.forward(Q, K, V, 1.04, 128, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)

@@ -124,6 +124,7 @@ struct Params {
   // the mask; the arithmetic is the router's, so the sets are identical
   int route_inkernel;
   int test_stall;       // failure-detection tests: the CTA's first S is never signalled
+  int out_align32;      // the output is 32-byte aligned: rows are written with 32-byte stores
   float scale;          // 1/sqrt(d) as the router computes it
   const float* qbar;    // [bH, Nq, d] fp32
   const float* kbar;    // [bH, Nk, d] fp32
@@ -146,8 +147,8 @@ struct Bars {
   uint64_t p_full[2];     // [S buffer]: both column halves have written P over S
   uint64_t o_full, o_free;
   uint64_t item_full[2], item_empty[2];
-  uint64_t xstate;        // softmax-state exchange between the halves at the end of an item
-  uint64_t xread;         // both halves have read the exchanged state
+  uint64_t xstate[4];     // [lane quadrant]: both halves' warps have written their row states
+  uint64_t xread[4];      // [lane quadrant]: both have read them (the rows may be rewritten)
   uint64_t teardown;
   int item_slot[2];
   int item_T[2];          // tiles of the item in each slot
@@ -380,8 +381,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars.item_full[s], 1);
       mbar_init(&bars.item_empty[s], 1 + SOFTMAX_WARPS);
     }
-    mbar_init(&bars.xstate, SOFTMAX_WARPS);
-    mbar_init(&bars.xread, SOFTMAX_WARPS);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bars.xstate[q], 2);
+      mbar_init(&bars.xread[q], 2);
+    }
     mbar_init(&bars.o_full, 1);
     mbar_init(&bars.o_free, SOFTMAX_WARPS);
     mbar_init(&bars.teardown, 1);
@@ -789,11 +792,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // e_h = 2^(m_h - max(m_0, m_1))
       // (one buffer: a half may finish the next item's key loop before its
       // partner has read this item's state, so writing waits for both reads)
-      if (item_local > 0 && !(ok = wait_warp(&bars.xread, (item_local - 1) & 1, bars, lim, 27))) break;
+      if (item_local > 0 && !(ok = wait_warp(&bars.xread[quad], (item_local - 1) & 1, bars, lim, 27))) break;
       bars.xm[half][row] = m_used;
       bars.xl[half][row] = l;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.xstate);
+      if (lane == 0) mbar_arrive(&bars.xstate[quad]);
       if (!(ok = wait_warp(&bars.o_full, item_local & 1, bars, lim, 24))) break;
       tc_fence_after();
       constexpr int OCH = C::OCHUNK;
@@ -807,30 +810,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.o_free);
-      if (!(ok = wait_warp(&bars.xstate, item_local & 1, bars, lim, 26))) break;
+      if (!(ok = wait_warp(&bars.xstate[quad], item_local & 1, bars, lim, 26))) break;
       const float m0 = bars.xm[0][row], m1 = bars.xm[1][row];
       const float mm = fmaxf(m0, m1);
       const float e0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
       const float e1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
       const float inv = 1.0f / (bars.xl[0][row] * e0 + bars.xl[1][row] * e1);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.xread);
+      if (lane == 0) mbar_arrive(&bars.xread[quad]);
       const float w0 = e0 * inv, w1 = e1 * inv;
       if (row < n_rows) {
+        // each thread writes its own row: one 32-byte store per 16 columns
+        // (a full sector) when the output allows it, else 16-byte stores
 #pragma unroll
         for (int q = 0; q < OCH; ++q) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            float v[8];
+          for (int c = 0; c < 32; c += 16) {
+            uint32_t w[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              v[e] = __uint_as_float(o0[q][c + e]) * w0 + __uint_as_float(o1[q][c + e]) * w1;
-            uint4 w;
-            w.x = pack_bf16x2(v[0], v[1]);
-            w.y = pack_bf16x2(v[2], v[3]);
-            w.z = pack_bf16x2(v[4], v[5]);
-            w.w = pack_bf16x2(v[6], v[7]);
-            *reinterpret_cast<uint4*>(orow + q * 32 + c) = w;
+              w[e] = pack_bf16x2(__uint_as_float(o0[q][c + 2 * e]) * w0 + __uint_as_float(o1[q][c + 2 * e]) * w1,
+                                 __uint_as_float(o0[q][c + 2 * e + 1]) * w0 +
+                                     __uint_as_float(o1[q][c + 2 * e + 1]) * w1);
+            if (p.out_align32) {
+              st_global_v8(orow + q * 32 + c, w);
+            } else {
+              *reinterpret_cast<uint4*>(orow + q * 32 + c) = make_uint4(w[0], w[1], w[2], w[3]);
+              *reinterpret_cast<uint4*>(orow + q * 32 + c + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+            }
           }
         }
       }
@@ -919,6 +926,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.chunks = correction ? g.nchunk : 0;
   p.route_inkernel = route_inkernel;
   p.test_stall = test_stall;
+  p.out_align32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   p.scale = 1.0f / sqrtf((float)g.d);  // the router's expression, evaluated the same way
   p.qbar = s.qbar; p.kbar = s.kbar; p.tau = s.tau;
   if (route_inkernel && (g.W > kInKernelMaxW || !s.tau)) return cudaErrorInvalidValue;
