@@ -53,7 +53,21 @@
 
 namespace sol {
 
-__device__ int g_sol_status;  // 0 = ok; else 0x1000 | wait id (first expiry)
+__device__ int g_sol_status;  // 0 = ok; else 0x1000 | wait id (first expiry), 0x3000 | check id
+
+// Consistency checks of the debug build (-DSOL_ATTN_DEBUG_CHECKS): a failed
+// check records its id in the status word (first failure wins) instead of
+// trapping, and the kernel carries on; the release build compiles them away.
+#ifdef SOL_ATTN_DEBUG_CHECKS
+#define SOL_DCHECK(cond, id)                                     \
+  do {                                                           \
+    if (!(cond)) atomicCAS(&g_sol_status, 0, 0x3000 | (id));     \
+  } while (0)
+#else
+#define SOL_DCHECK(cond, id) \
+  do {                       \
+  } while (0)
+#endif
 
 namespace {
 
@@ -236,6 +250,7 @@ struct TileIter {
 template <int HD>
 __device__ int route_row(const Params& p, int item, int lane, uint32_t& rb0, uint32_t& rb1) {
   const int bh = item / p.Nq;
+  SOL_DCHECK(p.W <= 64, 7);
   float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane * 4 < HD) qv = __ldg(reinterpret_cast<const float4*>(p.qbar + (size_t)item * HD) + lane);
   const float tau = __ldg(p.tau + item);
@@ -443,6 +458,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (item < 0) break;
       const int bh = item / p.Nq, qi = item % p.Nq;
+      SOL_DCHECK(item < p.nitems && bh < p.bH && T >= 0, 1);
       // the router's slot is released once this item's selection words are no
       // longer read (after its last tile is issued)
       auto release_route_slot = [&]() {
@@ -467,7 +483,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ++q_uses;
       for (int n = 0; n < T; ++n) {
         int kind = 0, tidx = 0, tidx2 = -1;
-        ti.next(kind, tidx, tidx2);
+        const bool has_tile = ti.next(kind, tidx, tidx2);
+        SOL_DCHECK(has_tile, 2);  // the item's tile count matches its selection
+        SOL_DCHECK(kind == 1 ? (tidx >= 0 && tidx < p.Nk && tidx2 < p.Nk && (p.pair || tidx2 < 0))
+                             : (tidx >= 0 && tidx < p.chunks),
+                   3);
         uint32_t vm[4] = {0u, 0u, 0u, 0u};
         if (kind == 0) {
 #pragma unroll
@@ -685,6 +705,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // the reads; the stage cannot refill before this warp hands over P
         if (!(ok = wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 22))) break;
         const int kind = bars.desc[ks].kind, tidx = bars.desc[ks].idx, tidx2 = bars.desc[ks].idx2;
+        SOL_DCHECK((kind == 0 && tidx < p.nchunk) || (kind == 1 && tidx < p.Nk && tidx2 < p.Nk), 4);
         tc_fence_after();
         float x[64];
         {
@@ -711,6 +732,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             nvalid = min(max(nblk - col0, 0), 64);
           }
         }
+        SOL_DCHECK(nvalid >= 0 && nvalid <= 64, 5);
         // full exact tile: x stays the raw score (scale folded into exp2 below);
         // otherwise x becomes the log2-domain logit with bias and mask applied
         const bool full = kind == 1 && nvalid == 64;
@@ -816,6 +838,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float e0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
       const float e1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
       const float inv = 1.0f / (bars.xl[0][row] * e0 + bars.xl[1][row] * e1);
+      SOL_DCHECK(inv > 0.f && inv < INFINITY, 6);  // every block with tiles has a positive row sum
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.xread[quad]);
       const float w0 = e0 * inv, w1 = e1 * inv;
