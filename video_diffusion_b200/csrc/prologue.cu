@@ -151,6 +151,8 @@ __global__ void __launch_bounds__(256) kvar_kernel(const float* __restrict__ kba
 
 constexpr int kRouteThreads = 256;
 constexpr int kRouteKC = 32;  // pooled keys staged in shared memory at a time
+template <int D>
+constexpr int route_ks_stride() { return D + 4; }  // 16-byte rows, and rows 4 banks apart
 
 // grid (ceil(Nq / QB), bH), 256 threads, QB a multiple of 8 (up to 32).
 // Score pass: lane l takes staged key l, warp w the query blocks
@@ -172,8 +174,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
   constexpr int QB = 8 * QPW;
   extern __shared__ float sm[];
   float* qs = sm;                          // [QB][D]
-  float* ks = qs + QB * D;                 // [KC][D + 1]
-  float* srow = ks + kRouteKC * (D + 1);   // [QB][Nk]
+  constexpr int KS = route_ks_stride<D>();
+  float* ks = qs + QB * D;                 // [KC][KS]
+  float* srow = ks + kRouteKC * KS;        // [QB][Nk]
   const int bh = blockIdx.y;
   const int i0 = blockIdx.x * QB;
   const int nq = min(QB, Nq - i0);
@@ -187,20 +190,29 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     __syncthreads();
     for (int e = tid; e < nk * D; e += kRouteThreads) {
       int jj = e / D, c = e % D;
-      ks[jj * (D + 1) + c] = kb[(size_t)(j0 + jj) * D + c];
+      ks[jj * KS + c] = kb[(size_t)(j0 + jj) * D + c];
     }
     __syncthreads();
     if (lane < nk) {
-      const float* kv = ks + lane * (D + 1);
+      const float* kv = ks + lane * KS;
       const float* qv = qs + warp * QPW * D;
       float acc[QPW];
 #pragma unroll
       for (int q = 0; q < QPW; ++q) acc[q] = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        const float kc = kv[c];
+      // four channels per 16-byte load (the query rows are broadcast to the
+      // warp); each sum still takes its channels in order, one fused
+      // multiply-add each, as the attention kernel's in-kernel routing does
+#pragma unroll 4
+      for (int c = 0; c < D; c += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kv + c);
 #pragma unroll
-        for (int q = 0; q < QPW; ++q) acc[q] = fmaf(qv[q * D + c], kc, acc[q]);
+        for (int q = 0; q < QPW; ++q) {
+          const float4 q4 = *reinterpret_cast<const float4*>(qv + q * D + c);
+          acc[q] = fmaf(q4.x, k4.x, acc[q]);
+          acc[q] = fmaf(q4.y, k4.y, acc[q]);
+          acc[q] = fmaf(q4.z, k4.z, acc[q]);
+          acc[q] = fmaf(q4.w, k4.w, acc[q]);
+        }
       }
 #pragma unroll
       for (int q = 0; q < QPW; ++q) {
@@ -239,39 +251,26 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     else tau = fmaf(beta, sigma, mu);
 
     const size_t item = (size_t)bh * Nq + i0 + qi;
-    int cnt = 0;
-    for (int w = lane; w < W; w += 32) {
-      uint32_t bits = 0;
-      const int jb = w * 32;
-      const int nb = min(32, Nk - jb);
-      for (int b = 0; b < nb; ++b) bits |= (s[jb + b] > tau ? 1u : 0u) << b;
-      if (mask) mask[item * W + w] = bits;
-      cnt += __popc(bits);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    // pooled-key chunks holding at least one unselected block
-    int used = 0;
-    if (correction) {
-      constexpr int wpc = kChunk / 32;  // mask words per chunk
-      for (int c = lane; c < nchunk; c += 32) {
-        bool any = false;
-        for (int q = 0; q < wpc; ++q) {
-          const int w = c * wpc + q;
-          if (w >= W) break;
-          const int jb = w * 32;
-          const int nb = min(32, Nk - jb);
-          const uint32_t valid = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
-          // recompute from scores: the words above may belong to other lanes
-          uint32_t bits = 0;
-          for (int b = 0; b < nb; ++b) bits |= (s[jb + b] > tau ? 1u : 0u) << b;
-          any |= ((~bits) & valid) != 0u;
-        }
-        used += any ? 1 : 0;
+    // one mask word per step: lane l tests key block 32w + l (consecutive
+    // shared-memory reads), a ballot gathers the word; a pooled-key chunk
+    // (kChunk / 32 words) counts as a tile if it holds an unselected block
+    constexpr int wpc = kChunk / 32;
+    int cnt = 0, used = 0;
+    bool chunk_has_unselected = false;
+    for (int w = 0; w < W; ++w) {
+      const int j = w * 32 + lane;
+      const bool valid = j < Nk;
+      const uint32_t word = __ballot_sync(0xffffffffu, valid && s[j] > tau);
+      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+      if (mask && lane == 0) mask[item * W + w] = word;
+      cnt += __popc(word);
+      chunk_has_unselected |= ((~word) & vmask) != 0u;
+      if (w % wpc == wpc - 1 || w == W - 1) {
+        used += chunk_has_unselected ? 1 : 0;
+        chunk_has_unselected = false;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) used += __shfl_xor_sync(0xffffffffu, used, o);
     }
+    if (!correction) used = 0;
     if (lane == 0) {
       counts[item] = cnt;
       tiles[item] = (pair ? (cnt + 1) >> 1 : cnt) + used;
@@ -359,7 +358,7 @@ template <int D, int QPW>
 static cudaError_t route_launch(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
                                 int pair, const float* kvar, cudaStream_t st) {
   constexpr int QB = 8 * QPW;
-  const size_t smem = (size_t)(QB * D + kRouteKC * (D + 1) + (size_t)QB * g.Nk) * sizeof(float);
+  const size_t smem = (size_t)(QB * D + kRouteKC * route_ks_stride<D>() + (size_t)QB * g.Nk) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(route_kernel<D, QPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((g.Nq + QB - 1) / QB, g.bH);
