@@ -468,31 +468,30 @@ def main():
         torch.cuda.synchronize()
         dense_ms = max_over_ranks(d0.elapsed_time(d1) / 2)
 
-    # end to end through the public call with host buffers
+    # end to end through the public call with host buffers: the library copies
+    # each group of heads in, computes it and copies it back, overlapped
     e2e = None
     if not args.no_e2e:
         hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
         hO = torch.empty_like(hQ).pin_memory()
-        dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(1, min(args.steps, 5))
+        api.forward_host(hQ, hK, hV, args.beta, blk, out=hO, diagonal_sigma=diag,
+                         route_in_kernel=args.route_in_kernel)  # warm-up: staging memory, internal streams
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(n_e2e):
-            dQ.copy_(hQ, non_blocking=True)
-            dK.copy_(hK, non_blocking=True)
-            dV.copy_(hV, non_blocking=True)
-            api.forward_ex(dQ, dK, dV, args.beta, blk, out=out, diagonal_sigma=diag,
-                           route_in_kernel=args.route_in_kernel)
-            hO.copy_(out, non_blocking=True)
+            api.forward_host(hQ, hK, hV, args.beta, blk, out=hO, diagonal_sigma=diag,
+                             route_in_kernel=args.route_in_kernel)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
         e2e = {"value": aggregate_value(world, wl.dense_flops(), e2e_ms), "unit": UNIT, "ms_per_call": e2e_ms,
                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
-               "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n_e2e}
-        del hQ, hK, hV, hO, dQ, dK, dV
+               "d2h_bytes_per_step": hO.numel() * hO.element_size(), "steps": n_e2e,
+               "call": "sol_attn_forward_host (pinned host buffers, copies overlapped with compute)"}
+        del hQ, hK, hV, hO
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -164,10 +164,36 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
                              int batch, int heads, int L, int d, int Bq, int Bk,
                              float beta, void* stream);
 
+/*
+ * Forward with the tensors in HOST memory: q, k, v are read from and out is
+ * written to host buffers (page-locked memory, e.g. from cudaHostAlloc, lets
+ * the copies run asynchronously; pageable memory works, with copies that
+ * block the host).  The paper has no counterpart: this is for callers that
+ * keep activations in host memory.  The (batch, head) slices are independent,
+ * so the call cuts them into groups of `slices_per_step` and pipelines the
+ * groups through two device staging buffers: group c + 1's inputs are copied
+ * in and group c - 1's output copied back (on two streams the library owns
+ * per device) while group c is computed on `stream`.  Same kernels and, slice
+ * for slice, the same results as sol_attn_forward_ex on device copies.
+ *   q, k, v        : const host pointers [batch, heads, L, d] of `dtype`, 16-byte aligned
+ *   out            : host pointer, same layout; complete once `stream` reaches
+ *                    the point where this call was enqueued
+ *   dtype, flags   : as sol_attn_forward_ex
+ *   slices_per_step: (batch, head) slices per group; 0 lets the library choose
+ *                    (about 8 groups, at most 1 GiB of staging); < 0 is
+ *                    SOL_ERR_INVALID_ARG
+ * The host buffers must stay valid and unmodified until then.  Staging (two
+ * groups of q, k, v and out) and scratch come stream-ordered from the
+ * library's pool, as for sol_attn_forward.  Errors as sol_attn_forward_ex.
+ */
+int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out, int dtype,
+                          int batch, int heads, int L, int d, int Bq, int Bk,
+                          float beta, unsigned int flags, int slices_per_step, void* stream);
+
 /* Human-readable name of a sol_status value. */
 const char* sol_attn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor): 103. */
+/* Library ABI version (major * 100 + minor): 104. */
 int sol_attn_version(void);
 
 #ifdef __cplusplus

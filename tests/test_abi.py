@@ -39,7 +39,7 @@ def test_status_strings_and_version(L):
     assert api.status_string(-1) == "SOL_ERR_INVALID_ARG"
     assert api.status_string(-5) == "SOL_ERR_DEVICE_TIMEOUT"
     assert api.status_string(7) == "SOL_ERR_UNKNOWN"
-    assert api.version() == 103
+    assert api.version() == 104
 
 
 # Argument checks run on the host before any CUDA call, so fake device
@@ -83,6 +83,26 @@ def test_stats_and_ex_reject_bad_arguments(L):
     assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 64 * 2049, 128, 128, 64, f(1.0), 4, None,
                                  None) == -2
     assert L.sol_attn_forward_ex(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 256, 96, 128, 64, f(1.0), 3, None, None) == -2
+
+
+def test_forward_host_rejects_bad_arguments(L):
+    """The host-buffer entry point checks everything before its first CUDA call."""
+    f = ctypes.c_float
+
+    def call(q=FAKE, k=FAKE, v=FAKE, o=FAKE, dtype=0, b=1, h=2, n=256, d=128, bq=128, bk=128, beta=1.0,
+             flags=0, g=0):
+        return L.sol_attn_forward_host(q, k, v, o, dtype, b, h, n, d, bq, bk, f(beta), flags, g, None)
+
+    assert call(q=0) == -1 and call(v=0) == -1 and call(o=0) == -1
+    assert call(k=FAKE + 4) == -1
+    assert call(dtype=3) == -1
+    assert call(flags=8) == -1
+    assert call(g=-1) == -1
+    assert call(beta=math.nan) == -1
+    assert call(h=0) == -1
+    assert call(d=80) == -2
+    assert call(bq=128, bk=32) == -2
+    assert call(dtype=1, flags=4) == -2  # in-kernel routing needs the tensor-core path
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

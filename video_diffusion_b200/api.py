@@ -24,8 +24,9 @@ FLAG_KEEP_OR_DROP = 1  # correction off: unselected blocks contribute nothing
 FLAG_DIAGONAL_SIGMA = 2  # sigma_i from the diagonal moment estimator
 FLAG_ROUTE_IN_KERNEL = 4  # Eq. 4 decided inside the attention kernel (no selection mask)
 
-EXPORTS = ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
-           "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_status_string", "sol_attn_version")
+EXPORTS = ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_forward_host",
+           "sol_attn_stats", "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_status_string",
+           "sol_attn_version")
 
 
 class SolAttnError(RuntimeError):
@@ -47,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L.sol_attn_forward_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, ctypes.c_uint,
                                           vp, vp]
         L.sol_attn_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
+        L.sol_attn_forward_host.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, ctypes.c_uint,
+                                            i32, vp]
         L.sol_attn_stats.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
         L.sol_attn_stats_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, ctypes.c_uint,
                                         vp]
@@ -56,7 +59,7 @@ def lib() -> ctypes.CDLL:
         L.sol_attn_version.argtypes = []
         for name in ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
                      "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_version",
-                     "sol_attn_forward_noalloc"):
+                     "sol_attn_forward_noalloc", "sol_attn_forward_host"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -139,10 +142,44 @@ def forward_ex(q, k, v, beta: float, block=128, out=None, events=None, stream=No
         ev = ctypes.cast(arr, ctypes.c_void_p)
     rc = lib().sol_attn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
                                    b, h, L, d, bq, bk, float(beta),
-                                   (FLAG_KEEP_OR_DROP if keep_or_drop else 0)
-                                   | (FLAG_DIAGONAL_SIGMA if diagonal_sigma else 0)
-                                   | (FLAG_ROUTE_IN_KERNEL if route_in_kernel else 0), ev, _stream_handle(stream))
+                                   _flags(keep_or_drop, diagonal_sigma, route_in_kernel), ev, _stream_handle(stream))
     _check("sol_attn_forward_ex", rc)
+    return out
+
+
+def _flags(keep_or_drop: bool, diagonal_sigma: bool, route_in_kernel: bool) -> int:
+    return ((FLAG_KEEP_OR_DROP if keep_or_drop else 0) | (FLAG_DIAGONAL_SIGMA if diagonal_sigma else 0)
+            | (FLAG_ROUTE_IN_KERNEL if route_in_kernel else 0))
+
+
+def forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, block=128,
+                 out: torch.Tensor | None = None, slices_per_step: int = 0, stream=None,
+                 keep_or_drop: bool = False, diagonal_sigma: bool = False,
+                 route_in_kernel: bool = False) -> torch.Tensor:
+    """forward() of [batch, heads, L, d] tensors in host memory (pin them for
+    overlapped copies): the library streams groups of (batch, head) slices
+    through device staging buffers on the current CUDA device, copying the
+    next group in and the previous group out while it computes.  `out` (a
+    host tensor) is complete once `stream` has reached this call; synchronise
+    it before reading."""
+    if q.dim() != 4:
+        raise ValueError("expected [batch, heads, L, d] tensors")
+    for t in (q, k, v):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v must share shape and dtype")
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous host tensors")
+    b, h, L, d = q.shape
+    bq, bk = blocks(block)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
+    if out.shape != q.shape or out.dtype != q.dtype or out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host tensor like q")
+    rc = lib().sol_attn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _dtype_code(q),
+                                     b, h, L, d, bq, bk, float(beta),
+                                     _flags(keep_or_drop, diagonal_sigma, route_in_kernel), int(slices_per_step),
+                                     _stream_handle(stream))
+    _check("sol_attn_forward_host", rc)
     return out
 
 

@@ -266,7 +266,7 @@ const char* sol_attn_status_string(int status) {
   }
 }
 
-int sol_attn_version(void) { return 103; }
+int sol_attn_version(void) { return 104; }
 
 }  // extern "C"
 
@@ -341,4 +341,128 @@ extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void
     e = sol::launch_attn_simt(0, q, k, v, out, g, s, st, 1);
   }
   return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------------- forward from host memory
+//
+// sol_attn_forward_host takes q, k, v and out in host memory.  The (batch,
+// head) slices are independent all the way through (pooling, routing and the
+// attention of one slice read nothing of another), so the call cuts them into
+// groups and pipelines the groups through two device staging buffers: while
+// group c is computed on the caller's stream, group c + 1's inputs are copied
+// in on one internal stream and group c - 1's output is copied back on
+// another.  Copy engines and SMs then work at the same time, and the call
+// takes about as long as its host-to-device copies.
+
+namespace {
+
+struct HostStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+};
+std::mutex g_host_mu;
+HostStreams g_host_streams[kMaxDevices];
+
+int host_streams(HostStreams* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SOL_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SOL_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostStreams& hs = g_host_streams[dev];
+  if (!hs.h2d && cudaStreamCreateWithFlags(&hs.h2d, cudaStreamNonBlocking) != cudaSuccess) return SOL_ERR_CUDA;
+  if (!hs.d2h && cudaStreamCreateWithFlags(&hs.d2h, cudaStreamNonBlocking) != cudaSuccess) return SOL_ERR_CUDA;
+  *out = hs;
+  return SOL_OK;
+}
+
+constexpr int kHostSteps = 8;                          // groups when the caller leaves the choice to the library
+constexpr size_t kHostStagingBytes = size_t(1) << 30;  // staging cap for the library's choice
+
+}  // namespace
+
+extern "C" int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out, int dtype, int batch,
+                                     int heads, int L, int d, int Bq, int Bk, float beta, unsigned int flags,
+                                     int slices_per_step, void* stream) {
+  if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
+  if (flags & ~(SOL_FLAG_KEEP_OR_DROP | SOL_FLAG_DIAGONAL_SIGMA | SOL_FLAG_ROUTE_IN_KERNEL))
+    return SOL_ERR_INVALID_ARG;
+  if (slices_per_step < 0) return SOL_ERR_INVALID_ARG;
+  Geometry g;
+  int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
+  if (rc != SOL_OK) return rc;
+  if ((flags & SOL_FLAG_ROUTE_IN_KERNEL) && (!uses_tensor_cores(dtype, g) || g.W > sol::kInKernelMaxW))
+    return SOL_ERR_UNSUPPORTED;
+  const size_t slice = (size_t)L * d * (dtype == SOL_DTYPE_BF16 ? 2 : 4);  // bytes of one (batch, head) slice
+  int G = slices_per_step;
+  if (G == 0) {
+    G = (g.bH + kHostSteps - 1) / kHostSteps;
+    const size_t cap = kHostStagingBytes / (8 * slice);  // two buffers of q, k, v, out
+    if ((size_t)G > cap) G = cap > 0 ? (int)cap : 1;
+  }
+  if (G > g.bH) G = g.bH;
+  const int steps = (g.bH + G - 1) / G;
+  const size_t group = slice * G;  // bytes of one tensor's group
+  HostStreams hs;
+  if ((rc = host_streams(&hs)) != SOL_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  cudaEvent_t ev[9] = {};  // start, in[2], comp[2], out[2], end[2]
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      for (auto& x : ev)
+        if (x) cudaEventDestroy(x);
+      cudaGetLastError();
+      return SOL_ERR_CUDA;
+    }
+  cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 3, *ev_out = ev + 5, *ev_end = ev + 7;
+  void* staging = nullptr;
+  if (scratch_alloc(&staging, 2 * 4 * group, st) != cudaSuccess) {
+    for (auto& x : ev) cudaEventDestroy(x);
+    cudaGetLastError();
+    return SOL_ERR_NO_MEMORY;
+  }
+  // staging buffer b: q, k, v, out groups back to back
+  auto buf = [&](int b, int t) { return static_cast<char*>(staging) + (size_t)(4 * b + t) * group; };
+  const char* hin[3] = {static_cast<const char*>(q), static_cast<const char*>(k), static_cast<const char*>(v)};
+  cudaError_t e = cudaEventRecord(ev_start, st);  // after the staging allocation and the caller's earlier work
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.h2d, ev_start, 0);
+  for (int c = 0; c < steps && e == cudaSuccess && rc == SOL_OK; ++c) {
+    const int b = c & 1;
+    const int n = c == steps - 1 ? g.bH - c * G : G;  // slices in this group
+    const size_t off = slice * (size_t)c * G, bytes = slice * n;
+    // inputs of group c, once group c - 2 no longer reads buffer b
+    if (c >= 2) e = cudaStreamWaitEvent(hs.h2d, ev_comp[b], 0);
+    for (int t = 0; t < 3 && e == cudaSuccess; ++t)
+      e = cudaMemcpyAsync(buf(b, t), hin[t] + off, bytes, cudaMemcpyHostToDevice, hs.h2d);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[b], hs.h2d);
+    // compute, once the inputs are in and group c - 2's output has left buffer b
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_in[b], 0);
+    if (e == cudaSuccess && c >= 2) e = cudaStreamWaitEvent(st, ev_out[b], 0);
+    if (e != cudaSuccess) break;
+    rc = forward_impl(buf(b, 0), buf(b, 1), buf(b, 2), buf(b, 3), dtype, 1, n, L, d, Bq, Bk, beta, flags, nullptr,
+                      st);
+    if (rc != SOL_OK) break;
+    e = cudaEventRecord(ev_comp[b], st);
+    // output of group c
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.d2h, ev_comp[b], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<char*>(out) + off, buf(b, 3), bytes, cudaMemcpyDeviceToHost, hs.d2h);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out[b], hs.d2h);
+  }
+  // the caller's stream goes on only after everything enqueued on the
+  // internal streams (every copy back, and any copy in left by an error):
+  // the staging memory is freed after them
+  for (int t = 0; t < 2; ++t) {
+    cudaStream_t is = t ? hs.d2h : hs.h2d;
+    cudaError_t e2 = cudaEventRecord(ev_end[t], is);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, ev_end[t], 0);
+    if (e == cudaSuccess) e = e2;
+  }
+  cudaFreeAsync(staging, st);
+  for (auto& x : ev) cudaEventDestroy(x);  // released once their pending records complete
+  if (rc != SOL_OK) return rc;
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SOL_ERR_CUDA;
+  }
+  return SOL_OK;
 }
