@@ -80,7 +80,7 @@ typedef enum {
  * Supported shapes: d in {64, 128}; Bq in {64, 128} and Bk in {64, 128}
  * (independently: query blocks of Bq tokens, key blocks of Bk tokens, the
  * Eq. 9 weight of a key block is its token count); L >= 1; batch * heads >= 1;
- * batch * heads * L * d < 2^40; ceil(L / Bk) <= 40960; beta not NaN.
+ * batch * heads * L * d < 2^40; ceil(L / Bk) <= 6144; beta not NaN.
  * Other values return SOL_ERR_UNSUPPORTED.  bf16 with Bq == 128 (any
  * supported d and Bk) runs the tensor-core (tcgen05/TMEM/TMA) kernel; every
  * other supported combination runs the CUDA-core kernel.

@@ -58,6 +58,7 @@ def call_fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, b=1, h=1, n=256, d=128, bq=128, 
     (dict(beta=float("nan")), -1),
     (dict(d=96), -2), (dict(d=256), -2), (dict(bq=96, bk=128), -2), (dict(bq=128, bk=32), -2),
     (dict(bq=32, bk=32), -2), (dict(bq=256, bk=256), -2), (dict(bq=128, bk=256), -2),
+    (dict(n=64 * 6145, bk=64), -2), (dict(n=128 * 6145), -2),
 ])
 def test_forward_rejects_bad_arguments(L, kw, code):
     assert call_fwd(L, **kw) == code

@@ -221,6 +221,23 @@ def test_video_workloads(name, beta, bk):
         assert 0.05 < frac < 0.30, frac
 
 
+# ------------------------------------------------------------------ many key blocks per head
+
+@pytest.mark.parametrize("grid,d,bk,diagonal", [
+    ((15, 100, 128), 128, 64, False),   # L = 192000, Nk = 3000: route_kernel, 8 score rows per CTA
+    ((15, 100, 128), 128, 64, True),
+    ((31, 100, 128), 64, 128, False),   # L = 396800, Nk = 3100 at d = 64: route_kernel
+    ((10, 100, 128), 128, 64, False),   # L = 128000, Nk = 2000: the register-blocked router
+    ((10, 100, 128), 128, 64, True),
+])
+def test_many_key_blocks(grid, d, bk, diagonal):
+    """Heads with more pooled keys than the register-blocked router's score
+    rows hold go through route_kernel; both must select what the oracle
+    selects, and the attention kernel must handle the long selection rows."""
+    Q, K, V = I.make_qkv(grid, heads=1, d=d, seed=41, device="cuda")
+    check_case(Q, K, V, (128, bk), 1.04, sample_k=4, seed=3, diagonal=diagonal)
+
+
 # ------------------------------------------------------------------ keep-or-drop (correction off)
 
 def check_keep_or_drop(Q, K, V, block, beta):

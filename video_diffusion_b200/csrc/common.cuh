@@ -42,7 +42,7 @@ struct Scratch {
   int32_t* work_counter;  // 1 int, zeroed before the attention kernel
 };
 
-constexpr int kRouteMaxN = 40960;   // pooled keys per head the router handles
+constexpr int kRouteMaxN = 6144;    // pooled keys per head the router handles (8 score rows in shared memory)
 constexpr int kOrderMaxN = 8192;    // query blocks per head the sorter handles
 
 // How sigma_i of Eq. 4 is estimated.

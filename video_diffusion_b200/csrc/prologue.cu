@@ -4,11 +4,12 @@
 //   "Pool Q, K and V into blocks" -> pool_kernel: Q-bar_i, K-bar_j are block
 //     means, V-hat_j the block sum (stored divided by n_j, with log n_j added to
 //     the pooled logit by the attention kernel: n_j e^a V-hat_j/n_j / (n_j e^a)).
-//   Eq. 4 / Eq. 5 -> route_kernel: the proxy row s_i = Q-bar_i K-bar^T / sqrt(d)
-//     is formed on chip (shared memory), its mean and population standard
-//     deviation give tau_i = mu_i + beta sigma_i, and S_i = {j : s_ij > tau_i}
+//   Eq. 4 / Eq. 5 -> route_blk_kernel (route_kernel for very long rows): the
+//     proxy row s_i = Q-bar_i K-bar^T / sqrt(d) is formed on chip (shared
+//     memory), and route_rows takes its mean and population standard
+//     deviation to tau_i = mu_i + beta sigma_i; S_i = {j : s_ij > tau_i}
 //     leaves as one bit per pair.  No Nq x Nk score map reaches global memory.
-//     The diagonal estimator named beside Eq. 5 (kvar_kernel + route_kernel)
+//     The diagonal estimator named beside Eq. 5 (kvar_kernel + route_rows)
 //     takes sigma_i from the per-channel variances of K-bar instead.
 // All reductions run in a fixed order, so results are deterministic.
 #include <cmath>
@@ -154,20 +155,85 @@ constexpr int kRouteKC = 32;  // pooled keys staged in shared memory at a time
 template <int D>
 constexpr int route_ks_stride() { return D + 4; }  // 16-byte rows, and rows 4 banks apart
 
-// grid (ceil(Nq / QB), bH), 256 threads, QB a multiple of 8 (up to 32).
-// Score pass: lane l takes staged key l, warp w the query blocks
-// w*QB/8 .. (w+1)*QB/8 - 1, so each thread runs QB/8 independent dot
-// products over one key row.  Row pass: warp w takes query blocks w, w + 8, ...
+// Row pass of the router for the score rows srow[qi * NS + j] (qi < nq,
+// j < Nk) of query blocks i0 .. i0 + nq - 1 of head bh: warp w of the
+// NTHREADS / 32 takes rows w, w + NTHREADS / 32, ...  qrows[qi * qstride ..] is Q-bar of row qi (diagonal estimator only).
 // kvar == nullptr: sigma_i from the row (Eq. 5); else the diagonal estimator.
 // tiles[i] counts the attention kernel's tiles: pooled-key chunks used plus the
 // selected blocks, two to a tile when pair != 0.  mask and tau_out may be null.
+template <int D, int NTHREADS>
+__device__ void route_rows(const float* srow, int NS, const float* qrows, int qstride, int bh, int i0, int nq,
+                           int Nq, int Nk,
+                           int W, float scale, float beta, int beta_mode, int correction, int pair,
+                           const float* __restrict__ kvar, uint32_t* __restrict__ mask,
+                           int32_t* __restrict__ counts, int32_t* __restrict__ tiles, float* __restrict__ tau_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int qi = warp; qi < nq; qi += NTHREADS / 32) {
+    const float* s = srow + (size_t)qi * NS;
+    // mean and population variance, two passes, lane-strided then a fixed tree
+    float a = 0.f;
+    for (int j = lane; j < Nk; j += 32) a += s[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    const float mu = a / (float)Nk;
+    float v = 0.f;
+    if (kvar == nullptr) {
+      for (int j = lane; j < Nk; j += 32) {
+        float t = s[j] - mu;
+        v = fmaf(t, t, v);
+      }
+    } else {
+      const float* qv = qrows + (size_t)qi * qstride;
+      const float* kvh = kvar + (size_t)bh * D;
+      for (int c = lane; c < D; c += 32) v = fmaf(qv[c] * qv[c], kvh[c], v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const float sigma = kvar == nullptr ? sqrtf(v / (float)Nk) : scale * sqrtf(v);
+    float tau;
+    if (beta_mode < 0) tau = -INFINITY;
+    else if (beta_mode > 0) tau = INFINITY;
+    else tau = fmaf(beta, sigma, mu);
+
+    const size_t item = (size_t)bh * Nq + i0 + qi;
+    // one mask word per step: lane l tests key block 32w + l (consecutive
+    // shared-memory reads), a ballot gathers the word; a pooled-key chunk
+    // (kChunk / 32 words) counts as a tile if it holds an unselected block
+    constexpr int wpc = kChunk / 32;
+    int cnt = 0, used = 0;
+    bool chunk_has_unselected = false;
+    for (int w = 0; w < W; ++w) {
+      const int j = w * 32 + lane;
+      const bool valid = j < Nk;
+      const uint32_t word = __ballot_sync(0xffffffffu, valid && s[j] > tau);
+      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+      if (mask && lane == 0) mask[item * W + w] = word;
+      cnt += __popc(word);
+      chunk_has_unselected |= ((~word) & vmask) != 0u;
+      if (w % wpc == wpc - 1 || w == W - 1) {
+        used += chunk_has_unselected ? 1 : 0;
+        chunk_has_unselected = false;
+      }
+    }
+    if (!correction) used = 0;
+    if (lane == 0) {
+      counts[item] = cnt;
+      tiles[item] = (pair ? (cnt + 1) >> 1 : cnt) + used;
+      if (tau_out) tau_out[item] = tau;
+    }
+  }
+}
+
+// Router for any Nk the shared memory holds at QB = 8 * QPW rows (up to 32).
+// grid (ceil(Nq / QB), bH), 256 threads.  Score pass: lane l takes staged key
+// l, warp w the query blocks w*QB/8 .. (w+1)*QB/8 - 1, so each thread runs
+// QB/8 independent dot products over one key row.
 template <int D, int QPW>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __restrict__ qbar,
                                                               const float* __restrict__ kbar,
                                                               const float* __restrict__ kvar, int Nq, int Nk,
-                                                              int W, int nchunk, float scale, float beta,
-                                                              int beta_mode, int correction, int pair,
-                                                              uint32_t* __restrict__ mask,
+                                                              int W, float scale, float beta, int beta_mode,
+                                                              int correction, int pair, uint32_t* __restrict__ mask,
                                                               int32_t* __restrict__ counts,
                                                               int32_t* __restrict__ tiles,
                                                               float* __restrict__ tau_out) {
@@ -222,61 +288,112 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     }
   }
   __syncthreads();
+  route_rows<D, kRouteThreads>(srow, Nk, qs, D, bh, i0, nq, Nq, Nk, W, scale, beta, beta_mode, correction, pair, kvar, mask,
+                counts, tiles, tau_out);
+}
 
-  for (int qi = warp; qi < nq; qi += kRouteThreads / 32) {
-    const float* s = srow + (size_t)qi * Nk;
-    // mean and population variance, two passes, lane-strided then a fixed tree
-    float a = 0.f;
-    for (int j = lane; j < Nk; j += 32) a += s[j];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    const float mu = a / (float)Nk;
-    float v = 0.f;
-    if (kvar == nullptr) {
-      for (int j = lane; j < Nk; j += 32) {
-        float t = s[j] - mu;
-        v = fmaf(t, t, v);
-      }
-    } else {
-      const float* qv = qs + qi * D;
-      const float* kvh = kvar + (size_t)bh * D;
-      for (int c = lane; c < D; c += 32) v = fmaf(qv[c] * qv[c], kvh[c], v);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    const float sigma = kvar == nullptr ? sqrtf(v / (float)Nk) : scale * sqrtf(v);
-    float tau;
-    if (beta_mode < 0) tau = -INFINITY;
-    else if (beta_mode > 0) tau = INFINITY;
-    else tau = fmaf(beta, sigma, mu);
+__device__ __forceinline__ void cp_async16(float* smem_dst, const float* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-    const size_t item = (size_t)bh * Nq + i0 + qi;
-    // one mask word per step: lane l tests key block 32w + l (consecutive
-    // shared-memory reads), a ballot gathers the word; a pooled-key chunk
-    // (kChunk / 32 words) counts as a tile if it holds an unselected block
-    constexpr int wpc = kChunk / 32;
-    int cnt = 0, used = 0;
-    bool chunk_has_unselected = false;
-    for (int w = 0; w < W; ++w) {
-      const int j = w * 32 + lane;
-      const bool valid = j < Nk;
-      const uint32_t word = __ballot_sync(0xffffffffu, valid && s[j] > tau);
-      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-      if (mask && lane == 0) mask[item * W + w] = word;
-      cnt += __popc(word);
-      chunk_has_unselected |= ((~word) & vmask) != 0u;
-      if (w % wpc == wpc - 1 || w == W - 1) {
-        used += chunk_has_unselected ? 1 : 0;
-        chunk_has_unselected = false;
-      }
+constexpr int kBlkThreads = 128;  // register-blocked router: four warps
+constexpr int kBlkQB = 16;        // query blocks per CTA
+constexpr int kBlkKC = 128;       // pooled keys staged per chunk (32 per warp)
+
+// Score-row stride of the register-blocked router: at least Nk and 8 banks
+// past a multiple of 32, so that the four rows a warp stores to at once fall
+// in different banks.
+__host__ __device__ inline int blk_row_stride(int Nk) { return Nk + ((8 - Nk) & 31); }
+
+// Router for Nk up to what 16 score rows leave room for (about 2400 pooled
+// keys at d = 128).  grid (ceil(Nq / 16), bH), 128 threads.  Score pass:
+// register-blocked like a small matrix product; lane (tq, tk) = (lane / 8,
+// lane % 8) of warp w computes query blocks tq + 4a (a < 4) against keys
+// 32w + tk + 8b (b < 4) of each staged chunk of 128, so per four channels it
+// makes 8 16-byte shared-memory loads (4 of query rows, 4 of key rows, each
+// shared by a group of lanes, conflict-free) for 64 fused multiply-adds.  Each
+// score is the same sequence of fused multiply-adds over the channels in
+// order, then the 1/sqrt(d) scale, as in route_kernel and the attention
+// kernel's in-kernel routing, so all three give the same bits.
+template <int D>
+__global__ void __launch_bounds__(kBlkThreads) route_blk_kernel(
+    const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ kvar, int Nq, int Nk,
+    int NS, int W, float scale, float beta, int beta_mode, int correction, int pair, uint32_t* __restrict__ mask,
+    int32_t* __restrict__ counts, int32_t* __restrict__ tiles, float* __restrict__ tau_out) {
+  constexpr int RS = route_ks_stride<D>();  // shared-memory row stride of Q-bar and K-bar rows
+  extern __shared__ __align__(16) float blk_sm[];
+  float* qs = blk_sm;                 // [16][RS]
+  float* ks = qs + kBlkQB * RS;       // [128][RS]
+  float* srow = ks + kBlkKC * RS;     // [16][NS]
+  const int bh = blockIdx.y;
+  const int i0 = blockIdx.x * kBlkQB;
+  const int nq = min(kBlkQB, Nq - i0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tq = lane >> 3, tk = lane & 7;
+  const float* qb = qbar + ((size_t)bh * Nq + i0) * D;
+  const float* kb = kbar + (size_t)bh * Nk * D;
+
+  // rows past nq repeat the last row; their scores are not stored
+  for (int e = tid; e < kBlkQB * (D / 4); e += kBlkThreads) {
+    const int r = e / (D / 4), c4 = e % (D / 4);
+    cp_async16(qs + r * RS + 4 * c4, qb + (size_t)min(r, nq - 1) * D + 4 * c4);
+  }
+  for (int j0 = 0; j0 < Nk; j0 += kBlkKC) {
+    const int nk = min(kBlkKC, Nk - j0);
+    __syncthreads();  // the previous chunk has been read by every warp
+    for (int e = tid; e < nk * (D / 4); e += kBlkThreads) {
+      const int r = e / (D / 4), c4 = e % (D / 4);
+      cp_async16(ks + r * RS + 4 * c4, kb + (size_t)(j0 + r) * D + 4 * c4);
     }
-    if (!correction) used = 0;
-    if (lane == 0) {
-      counts[item] = cnt;
-      tiles[item] = (pair ? (cnt + 1) >> 1 : cnt) + used;
-      if (tau_out) tau_out[item] = tau;
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    const int kw = warp * 32;  // this warp's 32 keys of the chunk
+    if (kw < nk) {
+      float acc[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+      const float* qr = qs + tq * RS;
+      const float* kr = ks + (kw + tk) * RS;  // key rows past nk hold stale data, never stored
+#pragma unroll 2
+      for (int c = 0; c < D; c += 4) {
+        float4 q4[4], k4[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) q4[a] = *reinterpret_cast<const float4*>(qr + 4 * a * RS + c);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) k4[b] = *reinterpret_cast<const float4*>(kr + 8 * b * RS + c);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            acc[a][b] = fmaf(q4[a].x, k4[b].x, acc[a][b]);
+            acc[a][b] = fmaf(q4[a].y, k4[b].y, acc[a][b]);
+            acc[a][b] = fmaf(q4[a].z, k4[b].z, acc[a][b]);
+            acc[a][b] = fmaf(q4[a].w, k4[b].w, acc[a][b]);
+          }
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const int qi = tq + 4 * a;
+        if (qi < nq) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int jj = kw + tk + 8 * b;
+            if (jj < nk) srow[(size_t)qi * NS + j0 + jj] = acc[a][b] * scale;
+          }
+        }
+      }
     }
   }
+  __syncthreads();
+  route_rows<D, kBlkThreads>(srow, NS, qs, RS, bh, i0, nq, Nq, Nk, W, scale, beta, beta_mode, correction, pair,
+                             kvar, mask, counts, tiles, tau_out);
 }
 
 // One CTA per head: bitonic sort of the head's work items by (tiles desc,
@@ -362,15 +479,32 @@ static cudaError_t route_launch(const Geometry& g, const Scratch& s, float beta,
   cudaError_t e = cudaFuncSetAttribute(route_kernel<D, QPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((g.Nq + QB - 1) / QB, g.bH);
-  route_kernel<D, QPW><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, g.W, g.nchunk,
+  route_kernel<D, QPW><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, g.W,
                                                           1.0f / sqrtf((float)D), beta, beta_mode, correction,
                                                           pair, s.mask, s.counts, s.tiles, s.tau);
   return cudaGetLastError();
 }
 
+constexpr size_t kRouteSmemMax = 227 * 1024;
+
+template <int D>
+static size_t route_blk_smem(int Nk) {
+  return (size_t)((kBlkQB + kBlkKC) * route_ks_stride<D>() + (size_t)kBlkQB * blk_row_stride(Nk)) * sizeof(float);
+}
+
 template <int D>
 static cudaError_t route_dispatch(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
                                  int pair, const float* kvar, cudaStream_t st) {
+  const size_t smem = route_blk_smem<D>(g.Nk);
+  if (smem <= kRouteSmemMax) {
+    cudaError_t e = cudaFuncSetAttribute(route_blk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((g.Nq + kBlkQB - 1) / kBlkQB, g.bH);
+    route_blk_kernel<D><<<grid, kBlkThreads, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, blk_row_stride(g.Nk),
+                                                        g.W, 1.0f / sqrtf((float)D), beta, beta_mode, correction,
+                                                        pair, s.mask, s.counts, s.tiles, s.tau);
+    return cudaGetLastError();
+  }
   const int qpw = route_qpw(g.Nk);
   if (qpw == 4) return route_launch<D, 4>(g, s, beta, beta_mode, correction, pair, kvar, st);
   if (qpw == 2) return route_launch<D, 2>(g, s, beta, beta_mode, correction, pair, kvar, st);
