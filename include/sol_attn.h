@@ -180,7 +180,7 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
  *                    the point where this call was enqueued
  *   dtype, flags   : as sol_attn_forward_ex
  *   slices_per_step: (batch, head) slices per group; 0 lets the library choose
- *                    (about 8 groups, at most 1 GiB of staging); < 0 is
+ *                    (about 16 groups, at most 1 GiB of staging); < 0 is
  *                    SOL_ERR_INVALID_ARG
  * The host buffers must stay valid and unmodified until then.  Staging (two
  * groups of q, k, v and out) and scratch come stream-ordered from the

@@ -238,6 +238,18 @@ def test_many_key_blocks(grid, d, bk, diagonal):
     check_case(Q, K, V, (128, bk), 1.04, sample_k=4, seed=3, diagonal=diagonal)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_largest_supported_key_block_count(d):
+    """Nk = 6144, the most pooled keys per head the library accepts (L = 393216
+    tokens in 64-token key blocks); one more block is rejected on the host."""
+    Q, K, V = I.make_qkv((24, 128, 128), heads=1, d=d, seed=42, device="cuda")
+    assert Q.shape[2] == 64 * 6144
+    check_case(Q, K, V, (128, 64), 1.04, sample_k=3, seed=4)
+    Q2 = torch.empty(1, 1, 64 * 6144 + 1, d, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(api.SolAttnError):
+        api.forward(Q2, Q2, Q2, 1.04, (128, 64))
+
+
 # ------------------------------------------------------------------ keep-or-drop (correction off)
 
 def check_keep_or_drop(Q, K, V, block, beta):

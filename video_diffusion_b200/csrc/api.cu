@@ -374,7 +374,7 @@ int host_streams(HostStreams* out) {
   return SOL_OK;
 }
 
-constexpr int kHostSteps = 8;                          // groups when the caller leaves the choice to the library
+constexpr int kHostSteps = 16;                         // groups when the caller leaves the choice to the library
 constexpr size_t kHostStagingBytes = size_t(1) << 30;  // staging cap for the library's choice
 
 }  // namespace
