@@ -265,7 +265,9 @@ def attention_kernel_name(wl, blk) -> str:
 
 
 def workload_key(wl, args) -> str:
-    key = f"{wl.name}_beta{args.beta:g}"
+    """File-name key of a workload's profile summaries: registry name, beta and
+    key block size when it differs from the query block."""
+    key = f"{args.workload}_beta{args.beta:g}"
     if args.block_k and args.block_k != wl.block:
         key += f"_bk{args.block_k}"
     return key

@@ -1,0 +1,65 @@
+"""Host-side pieces of bench.py that need no GPU: the profile lookup that
+fills roofline.traffic, and the executed-FLOP count the roofline divides."""
+
+import argparse
+import json
+import os
+
+import numpy as np
+
+import bench
+from video_diffusion_b200 import inputs as I
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _args(**kw):
+    a = dict(workload="wan-720p", beta=1.04, block_k=None)
+    a.update(kw)
+    return argparse.Namespace(**a)
+
+
+def test_default_workload_has_a_dram_profile_found_by_its_key():
+    """The default bench line looks up the DRAM capture of its own workload:
+    the key must name the committed summary file, and the record in it must
+    parse (its number is used while the kernel sources are unchanged)."""
+    wl = I.WORKLOADS["wan-720p"]
+    key = bench.workload_key(wl, _args())
+    assert key == "wan-720p_beta1.04"
+    path = os.path.join(ROOT, "profiles", f"attn_tc_kernel__{key}_dram.md")
+    assert os.path.exists(path)
+    recs = [json.loads(l) for l in open(path) if l.strip().startswith("{")]
+    assert len(recs) == 1
+    rec = recs[0]
+    assert rec["workload"] == "wan-720p" and rec["beta"] == 1.04
+    # about the algorithmic bytes of one launch: Q, K, V read and O written once
+    assert 3.0e9 < rec["dram_bytes_per_launch"] < 3.3e9
+    if rec["kernel_source_sha256"] == bench.kernel_source_digest():
+        assert bench.profiled_traffic(key) == rec["dram_bytes_per_launch"]
+    else:
+        assert bench.profiled_traffic(key) is None
+
+
+def test_workload_key_names_other_key_block_sizes():
+    wl = I.WORKLOADS["wan-720p"]
+    assert bench.workload_key(wl, _args(block_k=64)) == "wan-720p_beta1.04_bk64"
+    assert bench.workload_key(wl, _args(block_k=128)) == "wan-720p_beta1.04"
+    assert bench.profiled_traffic("no-such-workload_beta1") is None
+
+
+def test_executed_flops_counts_selected_pairs_and_pooled_columns():
+    """Three query and key blocks of 128, 128 and 64 tokens (L = 320), d = 2."""
+    sel = np.array([[True, False, True], [False, False, False], [True, True, True]])
+    d = 2
+    got = bench.executed_flops(sel[None, None], 320, 128, 128, d)
+    n = [128, 128, 64]
+    exact = sum(4 * n[i] * n[j] * d for i in range(3) for j in range(3) if sel[i, j])
+    # a query block with an unselected block scores all 3 pooled keys and
+    # folds in its unselected ones; block 2 selects everything and has no
+    # approximate work
+    unsel = [int((~sel[i]).sum()) for i in range(3)]
+    approx = sum(2 * n[i] * 3 * d + 2 * n[i] * unsel[i] * d for i in range(3) if unsel[i] > 0)
+    assert got["exact"] == exact
+    assert got["approx"] == approx
+    assert got["total"] == exact + approx
+    assert got["selected_fraction"] == sel.mean()
