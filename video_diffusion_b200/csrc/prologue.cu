@@ -300,52 +300,55 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-constexpr int kBlkThreads = 128;  // register-blocked router: four warps
-constexpr int kBlkQB = 16;        // query blocks per CTA
-constexpr int kBlkKC = 128;       // pooled keys staged per chunk (32 per warp)
+constexpr int kBlkKC = 128;  // register-blocked router: pooled keys staged per chunk (32 per warp)
 
 // Score-row stride of the register-blocked router: at least Nk and 8 banks
 // past a multiple of 32, so that the four rows a warp stores to at once fall
 // in different banks.
 __host__ __device__ inline int blk_row_stride(int Nk) { return Nk + ((8 - Nk) & 31); }
 
-// Router for Nk up to what 16 score rows leave room for (about 2400 pooled
-// keys at d = 128).  grid (ceil(Nq / 16), bH), 128 threads.  Score pass:
-// register-blocked like a small matrix product; lane (tq, tk) = (lane / 8,
-// lane % 8) of warp w computes query blocks tq + 4a (a < 4) against keys
-// 32w + tk + 8b (b < 4) of each staged chunk of 128, so per four channels it
+// Router for Nk up to what QH * 16 score rows leave room for (QH = 2: about
+// 1100 pooled keys at d = 128; QH = 1: about 2400).  grid (ceil(Nq / (16 QH)),
+// bH), 128 QH threads: QH groups of four warps, group h taking query blocks
+// 16h .. 16h + 15 of the CTA's.  Score pass: register-blocked like a small
+// matrix product; lane (tq, tk) = (lane / 8, lane % 8) of warp w of a group
+// computes its query blocks tq + 4a (a < 4) against keys 32w + tk + 8b (b < 4)
+// of each staged chunk of 128 (the chunk serves all QH groups), so per four
+// channels it
 // makes 8 16-byte shared-memory loads (4 of query rows, 4 of key rows, each
 // shared by a group of lanes, conflict-free) for 64 fused multiply-adds.  Each
 // score is the same sequence of fused multiply-adds over the channels in
 // order, then the 1/sqrt(d) scale, as in route_kernel and the attention
 // kernel's in-kernel routing, so all three give the same bits.
-template <int D>
-__global__ void __launch_bounds__(kBlkThreads) route_blk_kernel(
+template <int D, int QH>
+__global__ void __launch_bounds__(128 * QH) route_blk_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ kvar, int Nq, int Nk,
     int NS, int W, float scale, float beta, int beta_mode, int correction, int pair, uint32_t* __restrict__ mask,
     int32_t* __restrict__ counts, int32_t* __restrict__ tiles, float* __restrict__ tau_out) {
   constexpr int RS = route_ks_stride<D>();  // shared-memory row stride of Q-bar and K-bar rows
+  constexpr int QB = 16 * QH, NT = 128 * QH;
   extern __shared__ __align__(16) float blk_sm[];
-  float* qs = blk_sm;                 // [16][RS]
-  float* ks = qs + kBlkQB * RS;       // [128][RS]
-  float* srow = ks + kBlkKC * RS;     // [16][NS]
+  float* qs = blk_sm;                 // [QB][RS]
+  float* ks = qs + QB * RS;           // [128][RS]
+  float* srow = ks + kBlkKC * RS;     // [QB][NS]
   const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * kBlkQB;
-  const int nq = min(kBlkQB, Nq - i0);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i0 = blockIdx.x * QB;
+  const int nq = min(QB, Nq - i0);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int qg = tid >> 7, warp = (tid >> 5) & 3;  // query group, warp within the group
   const int tq = lane >> 3, tk = lane & 7;
   const float* qb = qbar + ((size_t)bh * Nq + i0) * D;
   const float* kb = kbar + (size_t)bh * Nk * D;
 
   // rows past nq repeat the last row; their scores are not stored
-  for (int e = tid; e < kBlkQB * (D / 4); e += kBlkThreads) {
+  for (int e = tid; e < QB * (D / 4); e += NT) {
     const int r = e / (D / 4), c4 = e % (D / 4);
     cp_async16(qs + r * RS + 4 * c4, qb + (size_t)min(r, nq - 1) * D + 4 * c4);
   }
   for (int j0 = 0; j0 < Nk; j0 += kBlkKC) {
     const int nk = min(kBlkKC, Nk - j0);
     __syncthreads();  // the previous chunk has been read by every warp
-    for (int e = tid; e < nk * (D / 4); e += kBlkThreads) {
+    for (int e = tid; e < nk * (D / 4); e += NT) {
       const int r = e / (D / 4), c4 = e % (D / 4);
       cp_async16(ks + r * RS + 4 * c4, kb + (size_t)(j0 + r) * D + 4 * c4);
     }
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kBlkThreads) route_blk_kernel(
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-      const float* qr = qs + tq * RS;
+      const float* qr = qs + (16 * qg + tq) * RS;
       const float* kr = ks + (kw + tk) * RS;  // key rows past nk hold stale data, never stored
 #pragma unroll 2
       for (int c = 0; c < D; c += 4) {
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(kBlkThreads) route_blk_kernel(
       }
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
-        const int qi = tq + 4 * a;
+        const int qi = 16 * qg + tq + 4 * a;
         if (qi < nq) {
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
@@ -392,8 +395,8 @@ __global__ void __launch_bounds__(kBlkThreads) route_blk_kernel(
     }
   }
   __syncthreads();
-  route_rows<D, kBlkThreads>(srow, NS, qs, RS, bh, i0, nq, Nq, Nk, W, scale, beta, beta_mode, correction, pair,
-                             kvar, mask, counts, tiles, tau_out);
+  route_rows<D, NT>(srow, NS, qs, RS, bh, i0, nq, Nq, Nk, W, scale, beta, beta_mode, correction, pair, kvar, mask,
+                    counts, tiles, tau_out);
 }
 
 // One CTA per head: bitonic sort of the head's work items by (tiles desc,
@@ -488,23 +491,31 @@ static cudaError_t route_launch(const Geometry& g, const Scratch& s, float beta,
 constexpr size_t kRouteSmemMax = 227 * 1024;
 
 template <int D>
-static size_t route_blk_smem(int Nk) {
-  return (size_t)((kBlkQB + kBlkKC) * route_ks_stride<D>() + (size_t)kBlkQB * blk_row_stride(Nk)) * sizeof(float);
+static size_t route_blk_smem(int Nk, int qh) {
+  return (size_t)((16 * qh + kBlkKC) * route_ks_stride<D>() + (size_t)16 * qh * blk_row_stride(Nk)) * sizeof(float);
+}
+
+template <int D, int QH>
+static cudaError_t route_blk_launch(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
+                                    int pair, const float* kvar, cudaStream_t st) {
+  const size_t smem = route_blk_smem<D>(g.Nk, QH);
+  cudaError_t e = cudaFuncSetAttribute(route_blk_kernel<D, QH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((g.Nq + 16 * QH - 1) / (16 * QH), g.bH);
+  route_blk_kernel<D, QH><<<grid, 128 * QH, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, blk_row_stride(g.Nk),
+                                                        g.W, 1.0f / sqrtf((float)D), beta, beta_mode, correction,
+                                                        pair, s.mask, s.counts, s.tiles, s.tau);
+  return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t route_dispatch(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
                                  int pair, const float* kvar, cudaStream_t st) {
-  const size_t smem = route_blk_smem<D>(g.Nk);
-  if (smem <= kRouteSmemMax) {
-    cudaError_t e = cudaFuncSetAttribute(route_blk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid((g.Nq + kBlkQB - 1) / kBlkQB, g.bH);
-    route_blk_kernel<D><<<grid, kBlkThreads, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, blk_row_stride(g.Nk),
-                                                        g.W, 1.0f / sqrtf((float)D), beta, beta_mode, correction,
-                                                        pair, s.mask, s.counts, s.tiles, s.tau);
-    return cudaGetLastError();
-  }
+  if (route_blk_smem<D>(g.Nk, 2) <= kRouteSmemMax)
+    return route_blk_launch<D, 2>(g, s, beta, beta_mode, correction, pair, kvar, st);
+  if (route_blk_smem<D>(g.Nk, 1) <= kRouteSmemMax)
+    return route_blk_launch<D, 1>(g, s, beta, beta_mode, correction, pair, kvar, st);
   const int qpw = route_qpw(g.Nk);
   if (qpw == 4) return route_launch<D, 4>(g, s, beta, beta_mode, correction, pair, kvar, st);
   if (qpw == 2) return route_launch<D, 2>(g, s, beta, beta_mode, correction, pair, kvar, st);
