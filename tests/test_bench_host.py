@@ -63,3 +63,36 @@ def test_executed_flops_counts_selected_pairs_and_pooled_columns():
     assert got["approx"] == approx
     assert got["total"] == exact + approx
     assert got["selected_fraction"] == sel.mean()
+
+
+def _run_bench(*argv, env_extra=None):
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *argv], capture_output=True, text=True,
+                          env=env, timeout=600, cwd=ROOT)
+
+
+def test_reference_arm_prints_one_oracle_line():
+    """`bench.py --impl reference` times the float64 oracle on the host (no
+    GPU) and prints the contract's line with the oracle as its baseline."""
+    p = _run_bench("--impl", "reference", "--workload", "tiny-fp32", "--steps", "2", "--warmup", "3")
+    assert p.returncode == 0, p.stderr
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["value"] > 0 and d["unit"] == bench.UNIT and d["metric"] == bench.METRIC
+    assert d["higher_is_better"] is True and d["dtype"] == "f64"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == I.WORKLOADS["tiny-fp32"].name
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    p = _run_bench("--impl", "reference", "--workload", "tiny-fp32", "--steps", "1",
+                   env_extra={"RANK": "1", "WORLD_SIZE": "2"})
+    assert p.returncode == 0, p.stderr
+    assert not [l for l in p.stdout.splitlines() if l.startswith("{")]
