@@ -178,9 +178,11 @@ def test_invalid_arguments_raise():
 @pytest.mark.parametrize("beta", [0.5, 1.04, 1.5])
 @pytest.mark.parametrize("name,bk", [("image-dit", 128), ("image-dit-d64", 128), ("image-dit-d64", 64)])
 def test_image_dit(beta, name, bk):
+    """The image-DiT workloads (24 heads, L = 16384) on every output row: the
+    oracle takes about half a second per head here."""
     wl = I.WORKLOADS[name]
     Q, K, V = I.make_workload(wl, device="cuda")
-    check_case(Q, K, V, (wl.block, bk), beta, sample_k=3, heads=range(wl.heads), seed=1)
+    check_case(Q, K, V, (wl.block, bk), beta)
 
 
 @pytest.mark.parametrize("name,beta,bk", [("wan-480p", 1.04, 128),
