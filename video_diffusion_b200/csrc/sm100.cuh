@@ -106,7 +106,7 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
-// 3-D tiled load (no multicast) into this CTA's shared memory; completion is
+// 3-D tiled load into this CTA's own shared memory only; completion is
 // signalled as transaction bytes on `bar`.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z,
                                             uint64_t cache_hint) {
