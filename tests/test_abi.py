@@ -112,3 +112,28 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(api, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         api.lib()
+
+
+def test_binding_rejects_bad_tensors_before_calling_the_library():
+    """The Python binding checks layout, device and dtype itself (ValueError)
+    before anything reaches the C ABI."""
+    import torch
+    from video_diffusion_b200 import api
+    q = torch.zeros(1, 2, 256, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.forward(q, q, q, 1.0)  # host tensors to the device entry point
+    with pytest.raises(ValueError, match="batch, heads, L, d"):
+        api.forward(q[0], q[0], q[0], 1.0)
+    with pytest.raises(ValueError, match="share"):
+        api.forward_host(q, q, q[:, :, :128], 1.0)
+    with pytest.raises(ValueError, match="contiguous"):
+        api.forward_host(q.transpose(2, 3), q.transpose(2, 3), q.transpose(2, 3), 1.0)
+    with pytest.raises(ValueError, match="out"):
+        api.forward_host(q, q, q, 1.0, out=torch.zeros(1, 2, 256, 128, dtype=torch.float32))
+    assert api.blocks(128) == (128, 128) and api.blocks((128, 64)) == (128, 64)
+    words = torch.tensor([[0b101, 1 << 31]], dtype=torch.int64).to(torch.int32)
+    bits = api.unpack_mask(words, 40)
+    assert bits.shape == (1, 40)
+    assert bits[0, 0] and not bits[0, 1] and bits[0, 2] and not bits[0, 31] and not bits[0, 39]
+    words = torch.tensor([[0, -2147483648]], dtype=torch.int32)  # bit 31 of word 1 = block 63
+    assert api.unpack_mask(words, 64)[0, 63] and api.unpack_mask(words, 64).sum() == 1
