@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ms/attention call and dense-equiv TFLOP/s at beta=1.04; % bf16 tensor peak"
 UNIT = "TFLOP/s (dense-equivalent)"
+NEAR_TIE_MARGIN = 1e-3  # |s_ij - tau_i| below this: a near tie (either decision is correct)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
@@ -53,17 +54,15 @@ def kernel_source_digest() -> str:
 
 
 def profiled_traffic(workload_key: str):
-    """DRAM bytes per attention launch from the committed ncu summary of this
-    workload, or None if there is none or the kernel changed since."""
-    p = os.path.join(ROOT, "profiles", f"attn_tc_kernel__{workload_key}_dram.md")
+    """DRAM bytes per attention launch from the committed ncu record of this
+    workload (profiles/<kernel>__<key>_dram.json), or None if there is none
+    or the kernel changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", f"attn_tc_kernel__{workload_key}_dram.json")
     if not os.path.exists(p):
         return None
-    for line in open(p):
-        line = line.strip()
-        if line.startswith("{") and "dram_bytes_per_launch" in line:
-            rec = json.loads(line)
-            if rec.get("kernel_source_sha256") == kernel_source_digest():
-                return float(rec["dram_bytes_per_launch"])
+    rec = json.load(open(p))
+    if rec.get("kernel_source_sha256") == kernel_source_digest():
+        return float(rec["dram_bytes_per_launch"])
     return None
 
 
@@ -179,57 +178,124 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- oracle timing (host)
 
-def oracle_sample_time(wl, beta: float, n_blocks: int = 2, seed: int = 0, block_k=None, moments="eq5"):
-    """Times the float64 oracle on one head's pooling + routing and `n_blocks`
-    query blocks of attention, and extrapolates to the whole call."""
+def host_cores() -> int:
+    """Cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_head_task(task):
+    """One worker process, one head: builds that head's inputs (untimed),
+    then times the float64 oracle's pooling + routing of the whole head and
+    its attention for `n_blocks` query blocks.  BLAS runs on one thread."""
+    name, head_seed, beta, bq, bk, moments, n_blocks, block_seed = task
+    import torch as _torch
+    _torch.set_num_threads(1)
     from oracle import sol_attn as O
     from video_diffusion_b200 import inputs as I
-    Q, K, V = I.make_qkv(wl.grid, 1, wl.d, wl.seed + seed, 1, wl.text_tokens, wl.dtype, "cpu")
+    wl = I.WORKLOADS[name]
+    Q, K, V = I.make_qkv(wl.grid, 1, wl.d, head_seed, 1, wl.text_tokens, wl.dtype, "cpu")
     Qh, Kh, Vh = (t[0, 0].double().numpy() for t in (Q, K, V))
-    bq, bk = wl.block, block_k or wl.block
     t0 = time.perf_counter()
     r = O.route_head(Qh, Kh, bq, bk, beta, moments)
     Vhat = O.pool_blocks(Vh, r["kgeom"], "sum")
     t1 = time.perf_counter()
     N = r["qgeom"].n
-    rng = np.random.default_rng(seed)
+    rng = np.random.default_rng(block_seed)
     blocks = rng.choice(N, size=min(n_blocks, N), replace=False)
     scale = 1.0 / math.sqrt(wl.d)
     for i in blocks:
         s0, n = int(r["qgeom"].starts[i]), int(r["qgeom"].counts[i])
         O.attend_query_block(Qh[s0:s0 + n], Kh, Vh, r["kgeom"], r["Kbar"], Vhat, r["sel"][i], scale)
     t2 = time.perf_counter()
-    per_head_prologue = t1 - t0
-    per_block = (t2 - t1) / len(blocks)
-    total = wl.batch * wl.heads * (per_head_prologue + per_block * N)
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    sample = (f"1 head pooling+routing and {len(blocks)} of {N} query blocks, extrapolated to "
-              f"{wl.batch * wl.heads} heads x {N} blocks")
-    return total, cores, sample, float(r["sel"].mean())
+    return t1 - t0, (t2 - t1) / len(blocks), len(blocks), N, float(r["sel"].mean())
+
+
+class OracleTimer:
+    """Times the float64 oracle on the host as it would run one call: one
+    process per head (BLAS pinned to one thread in each), as many processes as
+    this process has cores.  One sample = one head per process, each timing
+    its head's pooling + routing and `n_blocks` of its query blocks; the
+    whole call is extrapolated from the per-head times:
+        call = ceil(heads / processes) * (route + Nq * block).
+    The pool is made with the spawn method (a forked pool can hang after CUDA
+    is initialised)."""
+
+    def __init__(self, wl_key: str, beta: float, bq: int, bk: int, moments: str):
+        import multiprocessing as mp
+        from video_diffusion_b200 import inputs as I
+        self.wl = I.WORKLOADS[wl_key]
+        self.key, self.beta, self.bq, self.bk, self.moments = wl_key, beta, bq, bk, moments
+        self.cores = host_cores()
+        self.procs = max(1, min(self.cores, self.wl.batch * self.wl.heads))
+        for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+            os.environ[var] = "1"
+        self.pool = mp.get_context("spawn").Pool(self.procs)
+
+    def sample(self, step: int, n_blocks: int) -> dict:
+        tasks = [(self.key, self.wl.seed + 97 * step + p, self.beta, self.bq, self.bk, self.moments, n_blocks,
+                  1000 * step + p) for p in range(self.procs)]
+        t0 = time.perf_counter()
+        res = self.pool.map(_oracle_head_task, tasks)
+        wall = time.perf_counter() - t0
+        route = statistics.mean(r[0] for r in res)
+        block = statistics.mean(r[1] for r in res)
+        N = res[0][3]
+        heads = self.wl.batch * self.wl.heads
+        call = math.ceil(heads / self.procs) * (route + N * block)
+        return {"wall_s": wall, "route_s_per_head": route, "block_s": block, "blocks_per_head": res[0][2],
+                "heads_sampled": len(res), "call_s_extrapolated": call, "selected_fraction": res[0][4]}
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+    def describe(self, n_blocks: int) -> str:
+        heads = self.wl.batch * self.wl.heads
+        return (f"float64 oracle, {self.procs} processes (one head each, 1 BLAS thread): per head its pooling + "
+                f"routing and {n_blocks} of {self.wl.n_blocks} query blocks timed; the call "
+                f"({heads} heads x {self.wl.n_blocks} blocks) extrapolated as ceil({heads}/{self.procs}) x "
+                f"(route + {self.wl.n_blocks} x block)")
 
 
 def run_reference(args, wl):
+    """The reference arm: the oracle timed on the host's cores.  Each step is
+    one sample (one head per process, one query block each); `ms_per_step`
+    is that sample's measured wall time, while `value` is the whole call's
+    dense-equivalent rate extrapolated from the samples (marked so)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    times = []
-    for s in range(args.warmup + args.steps):
-        t, cores, sample, frac = oracle_sample_time(wl, args.beta, n_blocks=1, seed=s, block_k=args.block_k,
-                                                    moments=moments_of(args))
-        if s >= args.warmup:
-            times.append(t)
-    t = statistics.mean(times)
-    value = wl.dense_flops() / t / 1e12
+    bq, bk = blocks_of(wl, args)
+    timer = OracleTimer(args.workload, args.beta, bq, bk, moments_of(args))
+    samples = []
+    try:
+        for s in range(args.warmup + args.steps):
+            smp = timer.sample(s, n_blocks=1)
+            if s >= args.warmup:
+                samples.append(smp)
+    finally:
+        timer.close()
+    call_s = statistics.mean(x["call_s_extrapolated"] for x in samples)
+    wall_ms = statistics.mean(x["wall_s"] for x in samples) * 1e3
+    value = wl.dense_flops() / call_s / 1e12
+    sample = timer.describe(1)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(wl, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "extrapolated": True,
+        "timing": {"ms_per_step": "measured wall time of one sample (not of a whole call)",
+                   "value": "whole call, extrapolated from the samples",
+                   "call_s_extrapolated": call_s, "sample_wall_s": wall_ms / 1e3,
+                   "route_s_per_head": statistics.mean(x["route_s_per_head"] for x in samples),
+                   "block_s": statistics.mean(x["block_s"] for x in samples),
+                   "heads_per_sample": samples[0]["heads_sampled"], "blocks_per_head": 1},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": timer.procs, "kind": "oracle", "sample": sample,
+                         "extrapolated": True},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -345,6 +411,7 @@ def sweep_beta(args):
             out = dense
         counts, sel = api.stats(Q, K, beta, blk, with_mask=True, diagonal_sigma=diag)
         work = executed_flops(sel.cpu().numpy(), wl.L, blk[0], blk[1], wl.d)
+        near = int(api.near_ties(Q, K, beta, blk, margin=NEAR_TIE_MARGIN, diagonal_sigma=diag).sum())
         diff = out.float() - dref
         # the same beta with the correction off (keep-or-drop): what Eqs. 9-10 buy
         kod = torch.empty_like(Q)
@@ -354,6 +421,7 @@ def sweep_beta(args):
         kdiff = kod.float() - dref
         line = {"workload": wl.name, "block": list(blk), "sigma": moments_of(args), "beta": beta,
                 "selected_fraction": work["selected_fraction"],
+                "near_ties": near, "near_tie_margin": NEAR_TIE_MARGIN,
                 "gaussian_fraction": 0.5 * math.erfc(beta / math.sqrt(2)) if math.isfinite(beta) else
                 (1.0 if beta < 0 else 0.0),
                 "ms_per_call": ms, "dense_equiv_tflops": wl.dense_flops() / (ms * 1e-3) / 1e12,
@@ -424,6 +492,8 @@ def main():
     # selection statistics (same routing as the forward) for the FLOP count
     counts, sel = api.stats(Q, K, args.beta, blk, with_mask=True, diagonal_sigma=diag)
     work = executed_flops(sel.cpu().numpy(), wl.L, blk[0], blk[1], wl.d)
+    # decisions within 1e-3 of tau_i (where fp32 and fp64 routing may differ)
+    near = int(api.near_ties(Q, K, args.beta, blk, margin=NEAR_TIE_MARGIN, diagonal_sigma=diag).sum())
     del sel, counts
 
     for _ in range(args.warmup):
@@ -447,6 +517,8 @@ def main():
         torch.cuda.synchronize()
         clocks.mark_end()
     barrier()
+    # busy spread over the CTAs of the last timed attention launch
+    load_balance = api.load_balance(api.cta_times(stream))
     total_ms = start.elapsed_time(end)
     ms_step = max_over_ranks(total_ms / args.steps)
     stage = {"pool": [], "route": [], "attention": []}
@@ -457,18 +529,22 @@ def main():
     stage_ms = {k: statistics.mean(v) for k, v in stage.items()}
     clock_summary = clocks.summary()
 
-    # in-house dense comparator: the same kernel with beta = -inf
-    dense_ms = None
+    # in-house dense comparator: the same kernel with beta = -inf, timed like
+    # the sparse call (same warm-up, the same number of calls, at least 20)
+    dense_ms, dense_calls = None, 0
     if args.beta != -math.inf:
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        api.forward(Q, K, V, -math.inf, blk, out=out)
+        for _ in range(args.warmup):
+            api.forward(Q, K, V, -math.inf, blk, out=out)
+        dense_calls = max(args.steps, 20)
+        barrier()
         torch.cuda.synchronize()
         d0.record(stream)
-        for _ in range(2):
+        for _ in range(dense_calls):
             api.forward(Q, K, V, -math.inf, blk, out=out)
         d1.record(stream)
         torch.cuda.synchronize()
-        dense_ms = max_over_ranks(d0.elapsed_time(d1) / 2)
+        dense_ms = max_over_ranks(d0.elapsed_time(d1) / dense_calls)
 
     # end to end through the public call with host buffers: the library copies
     # each group of heads in, computes it and copies it back, overlapped
@@ -497,10 +573,14 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, cores, sample, _ = oracle_sample_time(wl, args.beta, n_blocks=2, block_k=args.block_k,
-                                                 moments=moments_of(args))
-        cpu = {"value": wl.dense_flops() / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": sample, "extrapolated_s_per_call": t}
+        timer = OracleTimer(args.workload, args.beta, blk[0], blk[1], moments_of(args))
+        try:
+            smp = timer.sample(0, n_blocks=2)
+        finally:
+            timer.close()
+        cpu = {"value": wl.dense_flops() / smp["call_s_extrapolated"] / 1e12, "unit": UNIT, "cores": timer.procs,
+               "kind": "oracle", "sample": timer.describe(2), "extrapolated": True,
+               "call_s_extrapolated": smp["call_s_extrapolated"], "sample_wall_s": smp["wall_s"]}
 
     attn_ms = max_over_ranks(stage_ms["attention"])
     achieved = work["total"] / (attn_ms * 1e-3) / 1e12
@@ -513,11 +593,15 @@ def main():
         "config": config_of(wl, args),
         "ms_per_call": ms_step,
         "selected_fraction": work["selected_fraction"],
+        "near_ties": {"margin": NEAR_TIE_MARGIN, "pairs": near,
+                      "fraction_of_pairs": near / float(wl.batch * wl.heads * wl.n_blocks * -(-wl.L // blk[1]))},
         "executed_tflop_per_call": work["total"] / 1e12,
         "executed_tflops": work["total"] / (ms_step * 1e-3) / 1e12,
         "pct_bf16_peak": 100.0 * work["total"] / (ms_step * 1e-3) / 1e12 / peak,
         "stages_ms": stage_ms,
+        "load_balance": load_balance,
         "dense_ms_per_call": dense_ms,
+        "dense_calls_timed": dense_calls,
         "speedup_vs_dense": (dense_ms / ms_step) if dense_ms else None,
         "target_speedup": 1.0 / (work["selected_fraction"] + 0.15),
         "roofline": {"kernel": attention_kernel_name(wl, blk), "bound": "tensor", "achieved": achieved,

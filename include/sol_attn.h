@@ -79,8 +79,9 @@ typedef enum {
 /*
  * Supported shapes: d in {64, 128}; Bq in {64, 128} and Bk in {64, 128}
  * (independently: query blocks of Bq tokens, key blocks of Bk tokens, the
- * Eq. 9 weight of a key block is its token count); L >= 1; batch * heads >= 1;
- * batch * heads * L * d < 2^40; ceil(L / Bk) <= 6144; beta not NaN.
+ * Eq. 9 weight of a key block is its token count); L >= 1;
+ * 1 <= batch * heads <= 65535; batch * heads * L * d < 2^40;
+ * ceil(L / Bk) <= 6144; beta not NaN.
  * Other values return SOL_ERR_UNSUPPORTED.  bf16 with Bq == 128 (any
  * supported d and Bk) runs the tensor-core (tcgen05/TMEM/TMA) kernel; every
  * other supported combination runs the CUDA-core kernel.
@@ -123,6 +124,25 @@ int sol_attn_stats_ex(const void* q, const void* k, int32_t* counts, uint32_t* m
                       float beta, int dtype, unsigned int flags, void* stream);
 
 /*
+ * Routing diagnostic: how many of each query block's decisions are near ties.
+ * Runs the forward's pooling and routing kernels (Eqs. 4-5) and writes, for
+ * every query block i,
+ *   near_ties[i] = #{ j : |s_ij - tau_i| < margin }      (s, tau as in Eq. 4)
+ * -- the pairs whose selection fp32 rounding may decide either way (an exact
+ * fp64 evaluation can land on the other side of tau_i).  With beta = +-INFINITY
+ * every count is 0.
+ *   near_ties: int32* [batch, heads, Nq] device
+ *   margin   : >= 0 and finite, in the units of s (logits scaled by 1/sqrt(d))
+ *   dtype, flags: as sol_attn_stats_ex (flags 0 or SOL_FLAG_DIAGONAL_SIGMA)
+ * The paper has no counterpart; it is a measurement aid.  Errors as
+ * sol_attn_stats (null near_ties or a negative, NaN or infinite margin:
+ * SOL_ERR_INVALID_ARG).
+ */
+int sol_attn_near_ties(const void* q, const void* k, int32_t* near_ties, float margin,
+                       int batch, int heads, int L, int d, int Bq, int Bk,
+                       float beta, int dtype, unsigned int flags, void* stream);
+
+/*
  * Extended forward.  Arguments as sol_attn_forward plus:
  *   dtype  : sol_dtype of q, k, v, out
  *   flags  : 0 or an OR of SOL_FLAG_KEEP_OR_DROP, SOL_FLAG_DIAGONAL_SIGMA,
@@ -139,9 +159,29 @@ int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, 
  * Reads and clears this device's status word, which a kernel sets when one of
  * its bounded waits runs out (it then abandons its work and exits cleanly).
  * Synchronises `stream` first.  Returns SOL_OK or SOL_ERR_DEVICE_TIMEOUT; if
- * detail is not NULL it receives the raw word (0 = no error).
+ * detail is not NULL it receives the raw word (0 = no error; else 0x1000 | the
+ * id of the first wait that ran out).
+ * There is ONE such word per device, shared by every call on every stream of
+ * the process: the first expiry since the last read is kept, later ones are
+ * dropped.  With calls in flight on several streams, the word cannot say
+ * which call's wait ran out; a caller that needs to know must read it after
+ * each call, with no other call of this library running on the device.
  */
 int sol_attn_device_status(void* stream, int32_t* detail);
+
+/*
+ * Load-balance record of the most recent tensor-core attention launch made by
+ * this process (on the current device): for each CTA of its grid (one per SM
+ * at most) one row of four uint64 -- start and end time of the CTA's work in
+ * ns of the GPU's global timer, the work items (query blocks) it took and the
+ * tiles it processed.  Synchronises `stream` first.  Writes min(grid,
+ * max_rows) rows to the host array `rows` and returns that count (0 if no
+ * such launch has been made), or a negative sol_status.  The record is one
+ * per device and the next tensor-core launch overwrites it; with launches in
+ * flight on several streams, read it with no other call running.  The paper
+ * has no counterpart: it is a measurement aid.
+ */
+int sol_attn_cta_times(void* stream, uint64_t* rows, int max_rows);
 
 /*
  * Forward without any memory allocation, for callers that may not allocate
@@ -152,7 +192,10 @@ int sol_attn_device_status(void* stream, int32_t* detail);
  *   - Scratch comes from a fixed 48 MiB device array inside the library,
  *     present on every GPU that loads it until the process exits.  A call
  *     whose scratch would not fit returns SOL_ERR_NO_MEMORY before enqueueing
- *     anything (the Wan2.1 720p and HunyuanVideo 720p calls fit).
+ *     anything.  With Bk = 128 the Wan2.1 720p call (40 heads, L = 75600)
+ *     needs about 37 MiB and the HunyuanVideo 720p call (24 heads,
+ *     L = 119056) about 36 MiB, so both fit; the same calls with Bk = 64 need
+ *     about 61 and 60 MiB and return SOL_ERR_NO_MEMORY.
  *   - The first call on a device looks up the array's device address (a
  *     cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls on a device share the array, and it keeps the previous call's
@@ -193,7 +236,7 @@ int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out
 /* Human-readable name of a sol_status value. */
 const char* sol_attn_status_string(int status);
 
-/* Library ABI version (major * 100 + minor): 104. */
+/* Library ABI version (major * 100 + minor): 105. */
 int sol_attn_version(void);
 
 #ifdef __cplusplus

@@ -21,17 +21,16 @@ def _args(**kw):
 
 def test_default_workload_has_a_dram_profile_found_by_its_key():
     """The default bench line looks up the DRAM capture of its own workload:
-    the key must name the committed summary file, and the record in it must
-    parse (its number is used while the kernel sources are unchanged)."""
+    the key must name the committed JSON record, which must parse (its
+    number is used while the kernel sources are unchanged)."""
     wl = I.WORKLOADS["wan-720p"]
     key = bench.workload_key(wl, _args())
     assert key == "wan-720p_beta1.04"
-    path = os.path.join(ROOT, "profiles", f"attn_tc_kernel__{key}_dram.md")
+    path = os.path.join(ROOT, "profiles", f"attn_tc_kernel__{key}_dram.json")
     assert os.path.exists(path)
-    recs = [json.loads(l) for l in open(path) if l.strip().startswith("{")]
-    assert len(recs) == 1
-    rec = recs[0]
+    rec = json.load(open(path))
     assert rec["workload"] == "wan-720p" and rec["beta"] == 1.04
+    assert "ncu" in rec["command"] and "--clock-control none" in rec["command"]
     # about the algorithmic bytes of one launch: Q, K, V read and O written once
     assert 3.0e9 < rec["dram_bytes_per_launch"] < 3.3e9
     if rec["kernel_source_sha256"] == bench.kernel_source_digest():
@@ -87,8 +86,35 @@ def test_reference_arm_prints_one_oracle_line():
     assert d["higher_is_better"] is True and d["dtype"] == "f64"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    # one head per process: the tiny workload has one head, so one process
+    assert cb["cores"] == 1 and cb["extrapolated"] is True and d["extrapolated"] is True
+    t = d["timing"]
+    assert t["heads_per_sample"] == 1 and t["blocks_per_head"] == 1
+    # ms_per_step is what was measured (one sample), the value is the call extrapolated
+    assert abs(d["ms_per_step"] - 1e3 * t["sample_wall_s"]) < 1e-6
+    assert t["call_s_extrapolated"] > 0 and t["route_s_per_head"] > 0 and t["block_s"] > 0
+    wl = I.WORKLOADS["tiny-fp32"]
+    assert abs(d["value"] - wl.dense_flops() / t["call_s_extrapolated"] / 1e12) <= 1e-9 * d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == I.WORKLOADS["tiny-fp32"].name
+
+
+def test_oracle_timer_extrapolates_one_call_from_per_head_times(monkeypatch):
+    """The extrapolation is ceil(heads / processes) x (route + Nq x block):
+    checked with a stand-in for the pool that returns fixed per-head times."""
+    class FakePool:
+        def map(self, fn, tasks):
+            return [(2.0, 0.5, 1, 591, 0.08) for _ in tasks]
+
+    t = bench.OracleTimer.__new__(bench.OracleTimer)
+    t.wl = I.WORKLOADS["wan-720p"]
+    t.key, t.beta, t.bq, t.bk, t.moments = "wan-720p", 1.04, 128, 128, "eq5"
+    t.cores, t.procs, t.pool = 16, 16, FakePool()
+    smp = t.sample(0, 1)
+    assert smp["heads_sampled"] == 16 and smp["blocks_per_head"] == 1
+    assert smp["call_s_extrapolated"] == 3 * (2.0 + 591 * 0.5)  # 40 heads on 16 processes: 3 rounds
+    assert "16 processes" in t.describe(1) and "ceil(40/16)" in t.describe(1)
+    assert bench.host_cores() >= 1
 
 
 def test_reference_arm_other_ranks_exit_quietly():

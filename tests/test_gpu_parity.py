@@ -348,3 +348,53 @@ def test_output_aligned_to_16_bytes_only(d):
     api.forward(Q, K, V, 1.04, 128, out=out)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+# ------------------------------------------------------------------ near-tie diagnostic
+
+@pytest.mark.parametrize("name,beta,margin", [("image-dit", 1.04, 1e-3), ("wan-480p", 0.5, 1e-2),
+                                              ("wan-480p", 1.04, 1e-3)])
+def test_near_tie_counts_match_the_oracle(name, beta, margin):
+    """sol_attn_near_ties counts, per query block, the key blocks whose proxy
+    score lies within `margin` of tau_i.  The GPU's scores and thresholds are
+    fp32 and the oracle's fp64, so a pair right at the margin may fall either
+    way: the count must lie between the oracle's counts at margin -/+ 1e-4."""
+    wl = I.WORKLOADS[name]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    near = api.near_ties(Q, K, beta, wl.block, margin=margin).cpu().numpy()
+    assert near.shape == (1, wl.heads, wl.n_blocks)
+    total = 0
+    for h in (0, wl.heads // 2, wl.heads - 1):
+        r = O.route_head(P.head_np(Q, 0, h), P.head_np(K, 0, h), wl.block, wl.block, beta)
+        gap = np.abs(r["s"] - r["tau"][:, None])
+        lo = (gap < margin - 1e-4).sum(axis=1)
+        hi = (gap < margin + 1e-4).sum(axis=1)
+        assert np.all(lo <= near[0, h]) and np.all(near[0, h] <= hi), h
+        total += int(near[0, h].sum())
+    assert total > 0  # the margins above catch some pairs on these workloads
+    for b in (-INF, INF):
+        assert not api.near_ties(Q, K, b, wl.block, margin=margin).any()
+
+
+def test_cta_times_account_for_every_item_and_tile():
+    """The per-CTA record of an attention launch covers the whole call: the
+    CTAs' item counts add up to batch x heads x Nq and their tile counts to
+    the selected blocks plus the pooled-key chunks that hold an unselected
+    block, per query block."""
+    wl = I.WORKLOADS["wan-480p"]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    api.forward(Q, K, V, 1.04, wl.block)
+    rows = api.cta_times()
+    counts, sel = api.stats(Q, K, 1.04, wl.block, with_mask=True)
+    sel = sel.cpu().numpy()
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    nitems = wl.heads * wl.n_blocks
+    assert len(rows) == min(n_sm, nitems)
+    assert np.all(rows[:, 1] > rows[:, 0])
+    assert rows[:, 2].sum() == nitems
+    Nk = sel.shape[-1]
+    chunks = -(-Nk // 128)
+    unsel_chunks = sum(((~sel[..., c * 128:(c + 1) * 128]).any(axis=-1)).sum() for c in range(chunks))
+    assert rows[:, 3].sum() == int(sel.sum()) + int(unsel_chunks)
+    lb = api.load_balance(rows)
+    assert 1.0 <= lb["busy_max_over_mean"] < 1.5 and 0.0 <= lb["tail_idle_fraction"] < 0.5

@@ -25,8 +25,8 @@ FLAG_DIAGONAL_SIGMA = 2  # sigma_i from the diagonal moment estimator
 FLAG_ROUTE_IN_KERNEL = 4  # Eq. 4 decided inside the attention kernel (no selection mask)
 
 EXPORTS = ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_forward_host",
-           "sol_attn_stats", "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_status_string",
-           "sol_attn_version")
+           "sol_attn_stats", "sol_attn_stats_ex", "sol_attn_near_ties", "sol_attn_cta_times", "sol_attn_device_status",
+           "sol_attn_status_string", "sol_attn_version")
 
 
 class SolAttnError(RuntimeError):
@@ -53,13 +53,17 @@ def lib() -> ctypes.CDLL:
         L.sol_attn_stats.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp]
         L.sol_attn_stats_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, ctypes.c_uint,
                                         vp]
+        L.sol_attn_near_ties.argtypes = [vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, f32, i32, ctypes.c_uint,
+                                         vp]
         L.sol_attn_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+        L.sol_attn_cta_times.argtypes = [vp, vp, i32]
         L.sol_attn_status_string.argtypes = [i32]
         L.sol_attn_status_string.restype = ctypes.c_char_p
         L.sol_attn_version.argtypes = []
         for name in ("sol_attn_forward", "sol_attn_forward_f32", "sol_attn_forward_ex", "sol_attn_stats",
                      "sol_attn_stats_ex", "sol_attn_device_status", "sol_attn_version",
-                     "sol_attn_forward_noalloc", "sol_attn_forward_host"):
+                     "sol_attn_forward_noalloc", "sol_attn_forward_host", "sol_attn_near_ties",
+                     "sol_attn_cta_times"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -86,6 +90,22 @@ def _shape(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor | None = None):
     return q.shape
 
 
+def _out_like(q: torch.Tensor, out: torch.Tensor | None) -> torch.Tensor:
+    """The output tensor: a new one like q, or the caller's after checking
+    that the kernels' row stores stay inside it (same shape, dtype and device
+    as q, contiguous CUDA memory)."""
+    if out is None:
+        return torch.empty_like(q)
+    if not isinstance(out, torch.Tensor):
+        raise ValueError("out must be a torch.Tensor")
+    if out.shape != q.shape or out.dtype != q.dtype or out.device != q.device:
+        raise ValueError(f"out must match q: shape {tuple(q.shape)}, dtype {q.dtype}, device {q.device} "
+                         f"(got {tuple(out.shape)}, {out.dtype}, {out.device})")
+    if not out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CUDA tensor")
+    return out
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return DTYPE_BF16
@@ -108,8 +128,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: float, bloc
     one size for query and key blocks or a (Bq, Bk) pair."""
     b, h, L, d = _shape(q, k, v)
     bq, bk = blocks(block)
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out_like(q, out)
     fn = lib().sol_attn_forward if q.dtype == torch.bfloat16 else lib().sol_attn_forward_f32
     _dtype_code(q)
     rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), b, h, L, d, bq, bk,
@@ -130,8 +149,7 @@ def forward_ex(q, k, v, beta: float, block=128, out=None, events=None, stream=No
     the attention kernel decide the selection itself (same results)."""
     b, h, L, d = _shape(q, k, v)
     bq, bk = blocks(block)
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out_like(q, out)
     ev = None
     if events is not None:
         arr = (ctypes.c_void_p * 4)()
@@ -204,11 +222,55 @@ def stats(q: torch.Tensor, k: torch.Tensor, beta: float, block=128, with_mask: b
     return counts, unpack_mask(mask, Nk)
 
 
+def near_ties(q: torch.Tensor, k: torch.Tensor, beta: float, block=128, margin: float = 1e-3, stream=None,
+              diagonal_sigma: bool = False) -> torch.Tensor:
+    """Per query block, the number of key blocks whose proxy score lies within
+    `margin` of the block's threshold tau_i ([batch, heads, Nq] int32)."""
+    b, h, L, d = _shape(q, k)
+    bq, bk = blocks(block)
+    near = torch.empty(b, h, -(-L // bq), dtype=torch.int32, device=q.device)
+    rc = lib().sol_attn_near_ties(q.data_ptr(), k.data_ptr(), near.data_ptr(), float(margin), b, h, L, d, bq, bk,
+                                  float(beta), _dtype_code(q), FLAG_DIAGONAL_SIGMA if diagonal_sigma else 0,
+                                  _stream_handle(stream))
+    _check("sol_attn_near_ties", rc)
+    return near
+
+
 def unpack_mask(words: torch.Tensor, N: int) -> torch.Tensor:
     """[..., W] int32 words -> [..., N] bool, bit j % 32 of word j // 32."""
     shifts = torch.arange(32, device=words.device, dtype=torch.int64)
     bits = (words.to(torch.int64).unsqueeze(-1) >> shifts) & 1
     return bits.reshape(*words.shape[:-1], words.shape[-1] * 32)[..., :N].bool()
+
+
+def cta_times(stream=None, max_rows: int = 1024):
+    """Per-CTA record of the last tensor-core attention launch: an int64
+    array [ctas, 4] of start ns, end ns, work items, tiles (synchronises)."""
+    import numpy as np
+    buf = np.zeros((max_rows, 4), dtype=np.uint64)
+    n = lib().sol_attn_cta_times(_stream_handle(stream), buf.ctypes.data, int(max_rows))
+    if n < 0:
+        _check("sol_attn_cta_times", n)
+    return buf[:n].astype(np.int64)
+
+
+def load_balance(rows) -> dict:
+    """Busy spread of one launch from cta_times(): per-CTA busy time
+    (end - start), its max / mean, and the tail-idle fraction = CTA time left
+    idle between each CTA's end and the last CTA's end, over all CTAs' span."""
+    import numpy as np
+    rows = np.asarray(rows, dtype=np.int64)
+    if len(rows) == 0:
+        return {}
+    t0, t1 = rows[:, 0].min(), rows[:, 1].max()
+    busy = (rows[:, 1] - rows[:, 0]).astype(np.float64)
+    span = float(t1 - t0)
+    return {"ctas": int(len(rows)), "span_ms": span * 1e-6, "busy_max_over_mean": float(busy.max() / busy.mean()),
+            "busy_min_over_mean": float(busy.min() / busy.mean()),
+            "tail_idle_fraction": float((t1 - rows[:, 1]).sum() / (span * len(rows))) if span > 0 else 0.0,
+            "start_skew_ms": float(rows[:, 0].max() - t0) * 1e-6,
+            "items_max_over_mean": float(rows[:, 2].max() / max(rows[:, 2].mean(), 1e-9)),
+            "tiles_max_over_mean": float(rows[:, 3].max() / max(rows[:, 3].mean(), 1e-9))}
 
 
 def device_status(stream=None) -> int:

@@ -31,7 +31,8 @@ int check_args(const void* q, const void* k, const void* v_or_dummy, const void*
   if (d != 64 && d != 128) return SOL_ERR_UNSUPPORTED;
   if ((Bq != 64 && Bq != 128) || (Bk != 64 && Bk != 128)) return SOL_ERR_UNSUPPORTED;
   const int64_t bH = (int64_t)batch * heads;
-  if (bH > (1 << 24) || bH * (int64_t)L * d >= (int64_t(1) << 40)) return SOL_ERR_UNSUPPORTED;
+  // batch * heads is the y dimension of the prologue kernels' grids
+  if (bH > sol::kMaxSlices || bH * (int64_t)L * d >= (int64_t(1) << 40)) return SOL_ERR_UNSUPPORTED;
   const int Nq = (L + Bq - 1) / Bq;
   const int Nk = (L + Bk - 1) / Bk;
   if (Nk > sol::kRouteMaxN) return SOL_ERR_UNSUPPORTED;
@@ -74,6 +75,8 @@ size_t carve(const Geometry& g, size_t op_elem, char* base, Scratch* s) {
   s->tiles = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
   s->order = reinterpret_cast<int32_t*>(take((size_t)g.nitems * sizeof(int32_t)));
   s->work_counter = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
+  s->near = nullptr;
+  s->near_margin = 0.f;
   return off;
 }
 
@@ -215,10 +218,16 @@ int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, 
                       static_cast<cudaStream_t>(stream));
 }
 
-int sol_attn_stats_ex(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int batch, int heads,
-                      int L, int d, int Bq, int Bk, float beta, int dtype, unsigned int flags, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Pooling and routing only (the forward's kernels, run the same way): counts
+// (and optionally the mask, or the near-tie counts) of every query block.
+int stats_impl(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int32_t* near,
+               float near_margin, int batch, int heads, int L, int d, int Bq, int Bk, float beta, int dtype,
+               unsigned int flags, void* stream) {
   if (dtype != SOL_DTYPE_BF16 && dtype != SOL_DTYPE_F32) return SOL_ERR_INVALID_ARG;
-  if (!counts) return SOL_ERR_INVALID_ARG;
   if (flags & ~SOL_FLAG_DIAGONAL_SIGMA) return SOL_ERR_INVALID_ARG;
   const int sigma_mode = (flags & SOL_FLAG_DIAGONAL_SIGMA) ? sol::kSigmaDiagonal : sol::kSigmaEq5;
   Geometry g;
@@ -233,13 +242,33 @@ int sol_attn_stats_ex(const void* q, const void* k, int32_t* counts, uint32_t* m
     return SOL_ERR_NO_MEMORY;
   }
   carve(g, 4, static_cast<char*>(base), &s);
-  s.counts = counts;
+  if (counts) s.counts = counts;
   if (mask_or_null) s.mask = mask_or_null;
+  s.near = near;
+  s.near_margin = near_margin;
   s.kbar_op = nullptr;  // routing needs the fp32 pooled vectors only
   cudaError_t e = sol::launch_pool(dtype == SOL_DTYPE_BF16 ? 0 : 1, 1, q, k, nullptr, g, s, st);
   if (e == cudaSuccess) e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, sigma_mode, 0, st);
   cudaFreeAsync(base, st);
   return e == cudaSuccess ? SOL_OK : SOL_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sol_attn_stats_ex(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int batch, int heads,
+                      int L, int d, int Bq, int Bk, float beta, int dtype, unsigned int flags, void* stream) {
+  if (!counts) return SOL_ERR_INVALID_ARG;
+  return stats_impl(q, k, counts, mask_or_null, nullptr, 0.f, batch, heads, L, d, Bq, Bk, beta, dtype, flags,
+                    stream);
+}
+
+int sol_attn_near_ties(const void* q, const void* k, int32_t* near_ties, float margin, int batch, int heads,
+                       int L, int d, int Bq, int Bk, float beta, int dtype, unsigned int flags, void* stream) {
+  if (!near_ties || !(margin >= 0.f) || std::isinf(margin)) return SOL_ERR_INVALID_ARG;
+  return stats_impl(q, k, nullptr, nullptr, near_ties, margin, batch, heads, L, d, Bq, Bk, beta, dtype, flags,
+                    stream);
 }
 
 int sol_attn_stats(const void* q, const void* k, int32_t* counts, uint32_t* mask_or_null, int batch, int heads,
@@ -254,6 +283,18 @@ int sol_attn_device_status(void* stream, int32_t* detail) {
   return w == 0 ? SOL_OK : SOL_ERR_DEVICE_TIMEOUT;
 }
 
+int sol_attn_cta_times(void* stream, uint64_t* rows, int max_rows) {
+  if (!rows || max_rows < 0) return SOL_ERR_INVALID_ARG;
+  int n = sol::last_attn_grid();
+  if (n > max_rows) n = max_rows;
+  if (n > sol::kMaxCtaTimes) n = sol::kMaxCtaTimes;
+  if (n == 0) return 0;
+  if (sol::read_cta_times(static_cast<cudaStream_t>(stream), reinterpret_cast<unsigned long long*>(rows), n) !=
+      cudaSuccess)
+    return SOL_ERR_CUDA;
+  return n;
+}
+
 const char* sol_attn_status_string(int status) {
   switch (status) {
     case SOL_OK: return "SOL_OK";
@@ -266,7 +307,7 @@ const char* sol_attn_status_string(int status) {
   }
 }
 
-int sol_attn_version(void) { return 104; }
+int sol_attn_version(void) { return 105; }
 
 }  // extern "C"
 
@@ -283,8 +324,10 @@ int sol_attn_version(void) { return 104; }
 namespace {
 
 // Fixed scratch, reserved on every GPU that loads this library until the
-// process exits.  48 MiB holds the scratch of the Wan2.1 720p call (40 heads,
-// L = 75600: about 38 MiB) and of the HunyuanVideo 720p call.
+// process exits.  At Bk = 128, 48 MiB holds the scratch of the Wan2.1 720p
+// call (40 heads, L = 75600: about 37 MiB) and of the HunyuanVideo 720p call
+// (about 36 MiB); with Bk = 64 those calls need about 61 and 60 MiB and are
+// refused with SOL_ERR_NO_MEMORY.
 constexpr size_t kNoAllocScratchBytes = size_t(48) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

@@ -55,6 +55,11 @@ namespace sol {
 
 __device__ int g_sol_status;  // 0 = ok; else 0x1000 | wait id (first expiry), 0x3000 | check id
 
+// Per-CTA record of the last attention launch on this device (a measurement
+// aid for load balance): start and end time (%globaltimer, ns), work items
+// and tiles the CTA processed.  Two timer reads and four stores per CTA.
+__device__ unsigned long long g_cta_times[kMaxCtaTimes][4];
+
 // Consistency checks of the debug build (-DSOL_ATTN_DEBUG_CHECKS): a failed
 // check records its id in the status word (first failure wins) instead of
 // trapping, and the kernel carries on; the release build compiles them away.
@@ -419,6 +424,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
+  const unsigned long long t_start = globaltimer_ns();
+  int n_items_done = 0, n_tiles_done = 0;  // producer's count, for the per-CTA record
 
   if (warp == 0) {
     // ================================================================ producer (whole warp, one lane issues)
@@ -466,6 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       if (T == 0) {
         release_route_slot();
+        ++n_items_done;
         continue;
       }
       // Q tile into buffer q_uses % QST, once the item that used it last has
@@ -534,6 +542,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!ok) break;
       release_route_slot();
       g += T;
+      ++n_items_done;
+      n_tiles_done += T;
     }
     if (!ok || bars.abort_flag) {
       // let every copy this warp started land before the CTA exits: the last
@@ -876,7 +886,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
+  if (threadIdx.x == 0 && blockIdx.x < kMaxCtaTimes) {
+    unsigned long long* rec = g_cta_times[blockIdx.x];
+    rec[0] = t_start;
+    rec[1] = globaltimer_ns();
+    rec[2] = (unsigned long long)n_items_done;
+    rec[3] = (unsigned long long)n_tiles_done;
+  }
 }
+
+int g_last_grid = 0;  // grid of the last tensor-core attention launch from this process
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -921,6 +940,7 @@ cudaError_t launch_hd(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtens
   if (e != cudaSuccess) return e;
   const int grid = nitems < nsm ? nitems : nsm;
   attn_tc_kernel<HD><<<grid, NTHREADS, smem, st>>>(mQ, mK, mV, mKb, mVb, p);
+  g_last_grid = grid;
   return cudaGetLastError();
 }
 
@@ -955,6 +975,15 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   if (route_inkernel && (g.W > kInKernelMaxW || !s.tau)) return cudaErrorInvalidValue;
   if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
   return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+}
+
+int last_attn_grid() { return g_last_grid; }
+
+cudaError_t read_cta_times(cudaStream_t st, unsigned long long* host, int n) {
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  if (n > kMaxCtaTimes) n = kMaxCtaTimes;
+  return cudaMemcpyFromSymbol(host, g_cta_times, (size_t)n * 4 * sizeof(unsigned long long));
 }
 
 cudaError_t read_device_status(cudaStream_t st, int32_t* word) {

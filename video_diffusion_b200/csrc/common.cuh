@@ -40,8 +40,13 @@ struct Scratch {
   int32_t* tiles;  // [bH, Nq]     tiles of the attention loop: |S_i| + pooled-key chunks used
   int32_t* order;  // [bH * Nq]    work items, head-major, heaviest first within a head
   int32_t* work_counter;  // 1 int, zeroed before the attention kernel
+  // routing diagnostics (null unless asked for): near[i] = number of key
+  // blocks j with |s_ij - tau_i| < near_margin
+  int32_t* near;
+  float near_margin;
 };
 
+constexpr int kMaxSlices = 65535;  // batch * heads: the prologue grids put it in gridDim.y
 constexpr int kRouteMaxN = 6144;    // pooled keys per head the router handles (8 score rows in shared memory)
 constexpr int kOrderMaxN = 8192;    // query blocks per head the sorter handles
 
@@ -73,5 +78,10 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
 cudaError_t launch_attn_simt(int dtype, const void* q, const void* k, const void* v, void* out,
                              const Geometry& g, const Scratch& s, cudaStream_t st, int correction);
 cudaError_t read_device_status(cudaStream_t st, int32_t* word);
+// Per-CTA record of the last tensor-core attention launch: n rows of
+// {start ns, end ns, items, tiles} (rows past the launch's grid are stale).
+constexpr int kMaxCtaTimes = 1024;
+cudaError_t read_cta_times(cudaStream_t st, unsigned long long* host, int n);
+int last_attn_grid();
 
 }  // namespace sol

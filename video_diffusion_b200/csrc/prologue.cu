@@ -166,7 +166,8 @@ __device__ void route_rows(const float* srow, int NS, const float* qrows, int qs
                            int Nq, int Nk,
                            int W, float scale, float beta, int beta_mode, int correction, int pair,
                            const float* __restrict__ kvar, uint32_t* __restrict__ mask,
-                           int32_t* __restrict__ counts, int32_t* __restrict__ tiles, float* __restrict__ tau_out) {
+                           int32_t* __restrict__ counts, int32_t* __restrict__ tiles, float* __restrict__ tau_out,
+                           int32_t* __restrict__ near, float near_margin) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int qi = warp; qi < nq; qi += NTHREADS / 32) {
     const float* s = srow + (size_t)qi * NS;
@@ -221,6 +222,13 @@ __device__ void route_rows(const float* srow, int NS, const float* qrows, int qs
       tiles[item] = (pair ? (cnt + 1) >> 1 : cnt) + used;
       if (tau_out) tau_out[item] = tau;
     }
+    if (near) {  // diagnostics only: decisions within near_margin of tau_i
+      int nt = 0;
+      for (int j = lane; j < Nk; j += 32) nt += fabsf(s[j] - tau) < near_margin ? 1 : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) nt += __shfl_xor_sync(0xffffffffu, nt, o);
+      if (lane == 0) near[item] = nt;
+    }
   }
 }
 
@@ -236,7 +244,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
                                                               int correction, int pair, uint32_t* __restrict__ mask,
                                                               int32_t* __restrict__ counts,
                                                               int32_t* __restrict__ tiles,
-                                                              float* __restrict__ tau_out) {
+                                                              float* __restrict__ tau_out,
+                                                              int32_t* __restrict__ near, float near_margin) {
   constexpr int QB = 8 * QPW;
   extern __shared__ float sm[];
   float* qs = sm;                          // [QB][D]
@@ -289,7 +298,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
   }
   __syncthreads();
   route_rows<D, kRouteThreads>(srow, Nk, qs, D, bh, i0, nq, Nq, Nk, W, scale, beta, beta_mode, correction, pair, kvar, mask,
-                counts, tiles, tau_out);
+                counts, tiles, tau_out, near, near_margin);
 }
 
 __device__ __forceinline__ void cp_async16(float* smem_dst, const float* gmem_src) {
@@ -324,7 +333,8 @@ template <int D, int QH>
 __global__ void __launch_bounds__(128 * QH) route_blk_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ kvar, int Nq, int Nk,
     int NS, int W, float scale, float beta, int beta_mode, int correction, int pair, uint32_t* __restrict__ mask,
-    int32_t* __restrict__ counts, int32_t* __restrict__ tiles, float* __restrict__ tau_out) {
+    int32_t* __restrict__ counts, int32_t* __restrict__ tiles, float* __restrict__ tau_out,
+    int32_t* __restrict__ near, float near_margin) {
   constexpr int RS = route_ks_stride<D>();  // shared-memory row stride of Q-bar and K-bar rows
   constexpr int QB = 16 * QH, NT = 128 * QH;
   extern __shared__ __align__(16) float blk_sm[];
@@ -396,7 +406,7 @@ __global__ void __launch_bounds__(128 * QH) route_blk_kernel(
   }
   __syncthreads();
   route_rows<D, NT>(srow, NS, qs, RS, bh, i0, nq, Nq, Nk, W, scale, beta, beta_mode, correction, pair, kvar, mask,
-                    counts, tiles, tau_out);
+                    counts, tiles, tau_out, near, near_margin);
 }
 
 // One CTA per head: bitonic sort of the head's work items by (tiles desc,
@@ -484,7 +494,8 @@ static cudaError_t route_launch(const Geometry& g, const Scratch& s, float beta,
   dim3 grid((g.Nq + QB - 1) / QB, g.bH);
   route_kernel<D, QPW><<<grid, kRouteThreads, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, g.W,
                                                           1.0f / sqrtf((float)D), beta, beta_mode, correction,
-                                                          pair, s.mask, s.counts, s.tiles, s.tau);
+                                                          pair, s.mask, s.counts, s.tiles, s.tau, s.near,
+                                                          s.near_margin);
   return cudaGetLastError();
 }
 
@@ -505,7 +516,8 @@ static cudaError_t route_blk_launch(const Geometry& g, const Scratch& s, float b
   dim3 grid((g.Nq + 16 * QH - 1) / (16 * QH), g.bH);
   route_blk_kernel<D, QH><<<grid, 128 * QH, smem, st>>>(s.qbar, s.kbar, kvar, g.Nq, g.Nk, blk_row_stride(g.Nk),
                                                         g.W, 1.0f / sqrtf((float)D), beta, beta_mode, correction,
-                                                        pair, s.mask, s.counts, s.tiles, s.tau);
+                                                        pair, s.mask, s.counts, s.tiles, s.tau, s.near,
+                                                        s.near_margin);
   return cudaGetLastError();
 }
 
