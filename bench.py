@@ -45,7 +45,7 @@ def kernel_source_digest() -> str:
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in ("attn_tc.cu", "sm100.cuh", "common.cuh"):
+    for f in ("attn_tc.cu", "attn_tc2.cuh", "sm100.cuh", "common.cuh"):
         text = open(os.path.join(ROOT, "video_diffusion_b200", "csrc", f)).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
@@ -435,6 +435,78 @@ def sweep_beta(args):
         del out, sel, counts, diff, kod, kdiff
 
 
+# ----------------------------------------------------------------------------- one call split by heads
+
+def run_sharded(args, wl, world, rank, local, dev, pg):
+    """One call of the workload split across the ranks by heads: `heads`
+    gives each rank its heads of every token; `ulysses` gives each rank its
+    token range of every head and times the seq -> head all-to-all of q, k
+    and v, the rank's heads, and the head -> seq all-to-all of the output.
+    The total work is fixed as N grows (strong scaling); timing is the max
+    over ranks of CUDA-event time on the launching stream."""
+    from video_diffusion_b200 import api
+    from video_diffusion_b200 import sharded as S
+    blk = blocks_of(wl, args)
+    Q, K, V = I_make(wl, dev)
+    counts, sel = api.stats(Q, K, args.beta, blk, with_mask=True)
+    work = executed_flops(sel.cpu().numpy(), wl.L, blk[0], blk[1], wl.d)
+    del counts, sel
+    if args.mode == "heads":
+        q, k, v = (S.shard_heads(t, world, rank).contiguous() for t in (Q, K, V))
+
+        def call():
+            return S.forward_heads(q, k, v, args.beta, blk)
+    else:
+        q, k, v = (S.shard_tokens(t, world, rank).contiguous() for t in (Q, K, V))
+
+        def call():
+            if pg is None:  # one rank: nothing to exchange
+                return api.forward(q, k, v, args.beta, blk)
+            return S.forward_ulysses(q, k, v, args.beta, wl.heads, wl.L, blk)
+    del Q, K, V
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        call()
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        clocks.mark_start()
+        e0.record(stream)
+        for _ in range(args.steps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark_end()
+    if pg is not None:
+        pg.barrier()
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, pg, dev)
+    heads_here = S.split_sizes(wl.heads, world)[rank]
+    line = {
+        "metric": METRIC, "value": wl.dense_flops() / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded smooth-field Q/K, V ~ N(0,1))",
+        "config": dict(config_of(wl, args), parallelism=f"{args.mode} x{world} (one call split by heads)"),
+        "ms_per_call": ms, "selected_fraction": work["selected_fraction"],
+        "executed_tflop_per_call": work["total"] / 1e12,
+        "heads_on_rank0": S.split_sizes(wl.heads, world)[0], "heads_here": heads_here,
+        "exchange_bytes_per_rank": (4 * S.exchange_bytes((wl.batch, wl.heads, wl.L, wl.d), 2, world, 0)
+                                    if args.mode == "ulysses" else 0),
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def I_make(wl, dev):
+    from video_diffusion_b200 import inputs as I
+    return I.make_workload(wl, device=dev)
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
@@ -453,6 +525,10 @@ def main():
                     help="let the attention kernel decide the selection itself (no selection mask)")
     ap.add_argument("--diagonal-sigma", action="store_true",
                     help="sigma_i of Eq. 4 from the diagonal moment estimator instead of Eq. 5")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "heads", "ulysses"],
+                    help="N > 1: replicas = one independent call per rank (weak scaling); heads = one call "
+                         "split across ranks by heads; ulysses = the same from sequence-sharded inputs, with "
+                         "the all-to-all re-layouts before and after (strong scaling)")
     ap.add_argument("--sweep-beta", default=None,
                     help="comma-separated betas: print one line per beta (fraction, time, speedup and "
                          "error against the beta=-inf output) instead of the benchmark line")
@@ -474,6 +550,11 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     pg = setup_dist(world, "nccl", dev)
+    if args.mode != "replicas":
+        run_sharded(args, wl, world, rank, local, dev, pg)
+        if pg is not None:
+            pg.destroy_process_group()
+        return
 
     def barrier():
         if pg is not None:
