@@ -47,6 +47,7 @@
 #include <cmath>
 #include <cstddef>
 #include <cstdint>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -895,6 +896,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+#include "attn_tc2.cuh"
+
 int g_last_grid = 0;  // grid of the last tensor-core attention launch from this process
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -944,6 +947,32 @@ cudaError_t launch_hd(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtens
   return cudaGetLastError();
 }
 
+template <int HD>
+cudaError_t launch_hd2(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtensorMap& mV, const CUtensorMap& mKb,
+                       const CUtensorMap& mVb, const Params& p, int nitems, cudaStream_t st) {
+  constexpr uint32_t smem = tc2::Cfg2<HD>::SMEM_BYTES;
+  int dev = 0, nsm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tc2::attn_tc2_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int want = (nitems + 1) / 2;  // two query blocks in flight per CTA
+  const int grid = want < nsm ? want : nsm;
+  tc2::attn_tc2_kernel<HD><<<grid, tc2::NTHREADS, smem, st>>>(mQ, mK, mV, mKb, mVb, p);
+  g_last_grid = grid;
+  return cudaGetLastError();
+}
+
+// SOL_ATTN_TWO_STREAM=1 selects the two-stream kernel (tc2::attn_tc2_kernel)
+// instead of the one-stream one (attn_tc_kernel, the default, faster as it
+// stands); both give the same results.
+bool one_stream_kernel() {
+  const char* e = std::getenv("SOL_ATTN_TWO_STREAM");
+  return !(e && *e && *e != '0');
+}
+
 }  // namespace
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
@@ -973,8 +1002,12 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.scale = 1.0f / sqrtf((float)g.d);  // the router's expression, evaluated the same way
   p.qbar = s.qbar; p.kbar = s.kbar; p.tau = s.tau;
   if (route_inkernel && (g.W > kInKernelMaxW || !s.tau)) return cudaErrorInvalidValue;
-  if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
-  return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+  if (one_stream_kernel()) {
+    if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+    return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+  }
+  if (g.d == 128) return launch_hd2<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+  return launch_hd2<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
 }
 
 int last_attn_grid() { return g_last_grid; }
