@@ -45,7 +45,7 @@ def kernel_source_digest() -> str:
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in ("attn_tc.cu", "attn_tc2.cuh", "sm100.cuh", "common.cuh"):
+    for f in ("attn_tc.cu", "sm100.cuh", "common.cuh"):
         text = open(os.path.join(ROOT, "video_diffusion_b200", "csrc", f)).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)

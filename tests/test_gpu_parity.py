@@ -398,33 +398,3 @@ def test_cta_times_account_for_every_item_and_tile():
     assert rows[:, 3].sum() == int(sel.sum()) + int(unsel_chunks)
     lb = api.load_balance(rows)
     assert 1.0 <= lb["busy_max_over_mean"] < 1.5 and 0.0 <= lb["tail_idle_fraction"] < 0.5
-
-
-# ------------------------------------------------------------------ the two-stream kernel
-
-@pytest.mark.parametrize("grid,heads,d,block,beta", [
-    ((5, 9, 40), 3, 128, 128, 1.04),           # L = 1800, ragged
-    ((5, 9, 40), 3, 128, 128, -INF),
-    ((4, 12, 20), 2, 128, (128, 64), 0.5),     # 64-token key blocks, two per tile
-    ((5, 9, 40), 3, 64, 128, 1.04),            # d = 64
-    ((3, 7, 30), 5, 128, 128, INF),            # everything through pooled keys
-])
-def test_two_stream_kernel_matches_oracle(monkeypatch, grid, heads, d, block, beta):
-    """SOL_ATTN_TWO_STREAM=1 runs the attention loop with two query blocks in
-    flight per CTA; it must pass the same parity checks."""
-    monkeypatch.setenv("SOL_ATTN_TWO_STREAM", "1")
-    Q, K, V = I.make_qkv(grid, heads=heads, d=d, seed=61, device="cuda")
-    check_case(Q, K, V, block, beta)
-
-
-def test_two_stream_kernel_is_bit_identical_run_to_run(monkeypatch):
-    monkeypatch.setenv("SOL_ATTN_TWO_STREAM", "1")
-    wl = I.WORKLOADS["wan-480p"]
-    Q, K, V = I.make_workload(wl, device="cuda")
-    a = api.forward(Q, K, V, 1.04, wl.block)
-    b = api.forward(Q, K, V, 1.04, wl.block)
-    assert torch.equal(a, b) and not torch.isnan(a).any()
-    monkeypatch.delenv("SOL_ATTN_TWO_STREAM")
-    one = api.forward(Q, K, V, 1.04, wl.block)
-    err = P.check_close(a.double().cpu().numpy(), one.double().cpu().numpy(), torch.bfloat16, "two vs one stream")
-    assert err["rel_l2"] < 5e-3

@@ -16,7 +16,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libsolattn.so")
 DEBUG_LIB = os.path.join(HERE, "libsolattn_debug.so")  # consistency checks on (tests only)
 SOURCES = ["api.cu", "prologue.cu", "attn_tc.cu", "attn_simt.cu"]
-HEADERS = ["common.cuh", "sm100.cuh", "attn_tc2.cuh"]
+HEADERS = ["common.cuh", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -455,7 +455,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         idx = __shfl_sync(0xffffffffu, idx, 0);
         item = idx < p.nitems ? p.order[idx] : -1;
         if (item >= 0) {
-          ti.init(p.mask + (size_t)item * p.W, p.W, p.Nk, p.chunks, p.pair);
+          const uint32_t* mrow = p.mask + (size_t)item * p.W;
+          if (p.W <= 64) {
+            // the item's selection row in two registers per lane (one
+            // coalesced load): walking its tiles then costs shuffles, not a
+            // dependent L2 round trip per mask word
+            ti.init(nullptr, p.W, p.Nk, p.chunks, p.pair);
+            ti.rb0 = lane < p.W ? __ldg(mrow + lane) : 0u;
+            ti.rb1 = 32 + lane < p.W ? __ldg(mrow + 32 + lane) : 0u;
+          } else {
+            ti.init(mrow, p.W, p.Nk, p.chunks, p.pair);
+          }
           T = p.tiles[item];
         }
       }
@@ -896,7 +906,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-#include "attn_tc2.cuh"
 
 int g_last_grid = 0;  // grid of the last tensor-core attention launch from this process
 
@@ -947,32 +956,6 @@ cudaError_t launch_hd(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtens
   return cudaGetLastError();
 }
 
-template <int HD>
-cudaError_t launch_hd2(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtensorMap& mV, const CUtensorMap& mKb,
-                       const CUtensorMap& mVb, const Params& p, int nitems, cudaStream_t st) {
-  constexpr uint32_t smem = tc2::Cfg2<HD>::SMEM_BYTES;
-  int dev = 0, nsm = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(tc2::attn_tc2_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  const int want = (nitems + 1) / 2;  // two query blocks in flight per CTA
-  const int grid = want < nsm ? want : nsm;
-  tc2::attn_tc2_kernel<HD><<<grid, tc2::NTHREADS, smem, st>>>(mQ, mK, mV, mKb, mVb, p);
-  g_last_grid = grid;
-  return cudaGetLastError();
-}
-
-// SOL_ATTN_TWO_STREAM=1 selects the two-stream kernel (tc2::attn_tc2_kernel)
-// instead of the one-stream one (attn_tc_kernel, the default, faster as it
-// stands); both give the same results.
-bool one_stream_kernel() {
-  const char* e = std::getenv("SOL_ATTN_TWO_STREAM");
-  return !(e && *e && *e != '0');
-}
-
 }  // namespace
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* out, const Geometry& g,
@@ -1002,12 +985,8 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.scale = 1.0f / sqrtf((float)g.d);  // the router's expression, evaluated the same way
   p.qbar = s.qbar; p.kbar = s.kbar; p.tau = s.tau;
   if (route_inkernel && (g.W > kInKernelMaxW || !s.tau)) return cudaErrorInvalidValue;
-  if (one_stream_kernel()) {
-    if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
-    return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
-  }
-  if (g.d == 128) return launch_hd2<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
-  return launch_hd2<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+  if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+  return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
 }
 
 int last_attn_grid() { return g_last_grid; }
