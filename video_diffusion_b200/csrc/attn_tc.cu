@@ -2,12 +2,14 @@
 // (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, d = 128 or 64,
 // query blocks of 128 tokens, key blocks of 128 or 64 tokens.
 //
-// What sets the pace is issue slots on the four schedulers, not the tensor
-// pipe: the softmax of a 128 x 128 tile takes about 900 issue slots per
-// scheduler, and the producer and MMA warps take theirs from the softmax
-// warps that share a scheduler with them.  So the control warps are kept
-// lean (descriptors built once, one commit per MMA group, waits that probe
-// before they block) and most exponentials go to the MUFU unit.
+// What sets the pace is the softmax of each tile and the round trip it
+// waits on: P of tile n is written over S in TMEM, so S of tile n + 2 can be
+// computed only after PV of tile n, and the softmax of a tile (max, 64
+// exponentials per thread, the bf16 P) is about as long as the tile's
+// tensor work.  The control warps are kept lean (descriptors built once, one
+// commit per MMA group, the selection row in registers, waits that probe
+// before they block), most exponentials go to the MUFU unit, and the merge
+// and store of each query block's output is left to a separate warpgroup.
 //
 // One online-softmax pass per query block i (Sol-Attn visual explainer, "One
 // online-softmax state": exact and approximate terms share the running
@@ -23,31 +25,37 @@
 //     128-column tile holds two selected blocks, one per softmax column half
 //     (an odd count leaves the last tile's second half masked out).
 //
-// Persistent CTAs, one per SM, 352 threads:
-//   warp 0      TMA producer: fetches work items, loads the Q tile and each
-//               tile's K and V (or K-bar and V-bar) together into a 3-stage
-//               ring (a tile copy takes about a tile's worth of time when
-//               every SM loads at once, so copies run up to three tiles ahead)
-//   warp 1      TMEM owner and tcgen05.mma issuer (one elected lane)
-//   warp 10     in-kernel routing only: fetches the work items and decides
-//               each one's selection ahead of the producer
-//   warps 2..9  softmax, two column halves: half h owns the 64 keys
-//               [64h, 64h + 64) of every tile, one query row per thread (its
-//               warp's TMEM lane quadrant).  Each half keeps its own running
-//               max, row sum and fp32 accumulator O_h = sum P_h V_h, so the
-//               halves never wait for each other inside the key loop; the two
-//               partial softmax states of a row are merged once per item.
+// Persistent CTAs, one per SM, 512 threads in four warpgroups (every
+// scheduler hosts one warp of each; the registers are rebalanced at start
+// with setmaxnreg: 72 per thread for the control warpgroup, 176 for the
+// softmax, 88 for the epilogue):
+//   warp 0        TMA producer: fetches work items, loads the Q tile and each
+//                 tile's K and V (or K-bar and V-bar) together into a 3-stage
+//                 ring (6 at d = 64)
+//   warp 1        TMEM owner and tcgen05.mma issuer (one elected lane)
+//   warp 2        in-kernel routing only: fetches the work items and decides
+//                 each one's selection ahead of the producer
+//   warps 4..11   softmax, two column halves: half h owns the 64 keys
+//                 [64h, 64h + 64) of every tile, one query row per thread (its
+//                 warp's TMEM lane quadrant).  Each half keeps its own running
+//                 max, row sum and fp32 accumulator O_h = sum P_h V_h, so the
+//                 halves never wait for each other inside the key loop; at the
+//                 end of a query block they leave their row states in shared
+//                 memory and go on with the next block.
+//   warps 12..15  epilogue: merge the two partial softmax states of each row
+//                 and write the output row (bf16), one row per thread.
 // TMEM columns: two S buffers [0,128) and [128,256) (tile n in buffer n % 2,
 // so S of the next tile is computed while the softmax works on this one; the
 // softmax writes P as bf16 pairs over the first 32 columns of each 64-column
-// half of its S), O_0 [256,384), O_1 [384,512).
+// half of its S), O_0 [256,384), O_1 [384,512).  At d = 64 an accumulator
+// takes 64 columns, so consecutive query blocks alternate between two banks
+// (O_h of bank b at 256 + 128 h + 64 b).
 // Every mbarrier wait is bounded; on expiry the CTA abandons its work, waits
 // for its own copies and MMAs, frees TMEM and records the failing wait in the
 // device status word.
 #include <cmath>
 #include <cstddef>
 #include <cstdint>
-#include <cstdlib>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -79,9 +87,21 @@ namespace {
 
 constexpr int BM = 128, BN = 128;
 constexpr int QST = 1;  // Q buffers
-constexpr int NTHREADS = 352;
-constexpr int ROUTER_WARP = 10;  // in-kernel routing: scores the items ahead of the producer
+// 16 warps in four warpgroups: control (producer, MMA, router, idle),
+// two softmax warpgroups (one per column half) and the epilogue warpgroup.
+// Warp w may access TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so every
+// warpgroup covers the four lane quadrants, and every scheduler (w % 4) hosts
+// one warp of each warpgroup.
+constexpr int NTHREADS = 512;
+constexpr int ROUTER_WARP = 2;  // in-kernel routing: scores the items ahead of the producer
 constexpr int SOFTMAX_WARPS = 8;
+constexpr int SOFTMAX_WARP0 = 4;  // warps 4..11: half (w - 4) / 4, quadrant w % 4
+constexpr int EPI_WARP0 = 12;     // warps 12..15: the epilogue, quadrant w % 4
+constexpr int EPI_WARPS = 4;
+// registers per thread after the warpgroups rebalance (setmaxnreg), within
+// the 64 K of the SM: 128 x 72 + 256 x 176 + 128 x 88 = 65536
+constexpr int REG_CONTROL = 72, REG_SOFTMAX = 176, REG_EPI = 88;
+static_assert(128 * REG_CONTROL + 256 * REG_SOFTMAX + 128 * REG_EPI <= 65536, "register split");
 constexpr uint32_t SLAB = BM * 128;  // 16 KB: 64 bf16 columns of a 128-row tile, 128-byte swizzled
 constexpr uint32_t BAR_AREA = 3072;
 
@@ -100,7 +120,6 @@ struct Cfg {
   static constexpr uint32_t OFF_KV = OFF_Q + QST * TILE_BYTES;  // stage s: K at +2s tiles, V at +2s+1
   static constexpr uint32_t OFF_BAR = OFF_KV + 2 * KVST * TILE_BYTES;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA;
-  static constexpr int OCHUNK = HD / 64;  // 32-column output chunks per softmax half
 };
 static_assert(Cfg<128>::SMEM_BYTES <= 227 * 1024 && Cfg<64>::SMEM_BYTES <= 227 * 1024, "shared memory");
 
@@ -108,16 +127,23 @@ static_assert(Cfg<128>::SMEM_BYTES <= 227 * 1024 && Cfg<64>::SMEM_BYTES <= 227 *
 // P overwrites the first 32 columns of each 64-column half, as bf16 pairs),
 // O_h at TM_O + 128 h
 constexpr uint32_t TM_S = 0, TM_O = 256;
+// O banks: at d = 64 an accumulator takes 64 of its half's 128 columns, so
+// consecutive items alternate between two banks and an item's PVs need not
+// wait for the previous item's epilogue to read O
+template <int HD>
+constexpr int o_banks() { return HD == 64 ? 2 : 1; }
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 // A share of the probabilities goes through an FMA-pipe polynomial exp2
-// instead of the MUFU ex2 unit: NPOLY of every 8 column pairs.  The softmax
-// warps are bound by issue slots rather than by MUFU throughput (4 lanes per
-// cycle per scheduler), above all on the schedulers that also host the
-// producer and the MMA warp, and the polynomial costs five times the issue
-// slots of MUFU: measured on Wan 720p, 0 or 1 of 8 is fastest, 3 of 8 about
-// 3 % slower.
-constexpr int NPOLY = 1;
+// instead of the MUFU ex2 unit: npoly<HD>() of every 8 column pairs.  At
+// d = 128 the softmax warps are bound by issue slots rather than by MUFU
+// throughput (4 lanes per cycle per scheduler), and the polynomial costs five
+// times the issue slots of MUFU: measured on Wan 720p, 0 to 4 of 8 lie within
+// the clock spread, 1 of 8 is kept.  At d = 64 a tile's tensor work halves
+// while its exponentials stay, MUFU sets the pace, and 3 of 8 measured fastest
+// (image-DiT d = 64, beta = 1.04: 0.325 of the measured peak against 0.310).
+template <int HD>
+constexpr int npoly() { return HD == 64 ? 3 : 1; }
 template <int NP>
 __host__ __device__ constexpr bool poly_pair(int pair) {
   return NP >= 3   ? ((pair & 7) == 2 || (pair & 7) == 5 || (pair & 7) == 7)
@@ -165,10 +191,10 @@ struct Bars {
   uint64_t kv_full[KVST], kv_empty[KVST];
   uint64_t s_full[2];     // [S buffer]: S of the buffer's tile is in TMEM
   uint64_t p_full[2];     // [S buffer]: both column halves have written P over S
-  uint64_t o_full, o_free;
+  uint64_t o_full[2], o_free[2];  // [O bank]: the item's last PV is done / the epilogue has read O
   uint64_t item_full[2], item_empty[2];
-  uint64_t xstate[4];     // [lane quadrant]: both halves' warps have written their row states
-  uint64_t xread[4];      // [lane quadrant]: both have read them (the rows may be rewritten)
+  uint64_t state_full;     // the softmax warps have left the item's row states
+  uint64_t state_empty;    // the epilogue has read them
   uint64_t teardown;
   int item_slot[2];
   int item_T[2];          // tiles of the item in each slot
@@ -400,14 +426,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.p_full[s], SOFTMAX_WARPS);
       mbar_init(&bars.item_full[s], 1);
-      mbar_init(&bars.item_empty[s], 1 + SOFTMAX_WARPS);
+      mbar_init(&bars.item_empty[s], 1 + SOFTMAX_WARPS + EPI_WARPS);
+      mbar_init(&bars.o_full[s], 1);
+      mbar_init(&bars.o_free[s], EPI_WARPS);
     }
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(&bars.xstate[q], 2);
-      mbar_init(&bars.xread[q], 2);
-    }
-    mbar_init(&bars.o_full, 1);
-    mbar_init(&bars.o_free, SOFTMAX_WARPS);
+    mbar_init(&bars.state_full, SOFTMAX_WARPS);
+    mbar_init(&bars.state_empty, EPI_WARPS);
     mbar_init(&bars.teardown, 1);
     for (int s = 0; s < 2; ++s) { mbar_init(&bars.rq_full[s], 1); mbar_init(&bars.rq_empty[s], 1); }
     bars.abort_flag = 0;
@@ -428,273 +452,357 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const unsigned long long t_start = globaltimer_ns();
   int n_items_done = 0, n_tiles_done = 0;  // producer's count, for the per-CTA record
 
-  if (warp == 0) {
-    // ================================================================ producer (whole warp, one lane issues)
-    const bool leader = elect_one();
-    const uint64_t pol_kv = policy_evict_last();
-    const uint64_t pol_q = policy_evict_first();
-    uint32_t g = 0;          // global tile counter
-    // last K / V tile and number of Q tiles whose loads were issued (to let
-    // them land if the CTA abandons its work)
-    int gk_last = -1, q_uses = 0;
-    bool ok = true;
-    for (int it = 0;; ++it) {
-      const int slot = it & 1;
-      if (it >= 2 && !(ok = wait_warp(&bars.item_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 1))) break;
-      int item = -1, T = 0;
-      TileIter ti;
-      if (p.route_inkernel) {
-        // the router warp has fetched and scored the item already
-        if (!(ok = wait_warp(&bars.rq_full[slot], (it >> 1) & 1, bars, lim, 4))) break;
-        item = bars.rq_item[slot];
-        T = bars.rq_T[slot];
-        ti.init(bars.rq_bits[slot], p.W, p.Nk, p.chunks, p.pair);
-      } else {
+  if (warp < 4) {
+    setmaxnreg_dec<REG_CONTROL>();
+    if (warp == 0) {
+      // ================================================================ producer (whole warp, one lane issues)
+      const bool leader = elect_one();
+      const uint64_t pol_kv = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
+      uint32_t g = 0;          // global tile counter
+      // last K / V tile and number of Q tiles whose loads were issued (to let
+      // them land if the CTA abandons its work)
+      int gk_last = -1, q_uses = 0;
+      bool ok = true;
+      for (int it = 0;; ++it) {
+        const int slot = it & 1;
+        if (it >= 2 && !(ok = wait_warp(&bars.item_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 1))) break;
+        int item = -1, T = 0;
+        TileIter ti;
+        if (p.route_inkernel) {
+          // the router warp has fetched and scored the item already
+          if (!(ok = wait_warp(&bars.rq_full[slot], (it >> 1) & 1, bars, lim, 4))) break;
+          item = bars.rq_item[slot];
+          T = bars.rq_T[slot];
+          ti.init(bars.rq_bits[slot], p.W, p.Nk, p.chunks, p.pair);
+        } else {
+          int idx = 0;
+          if (lane == 0) idx = atomicAdd(p.work_counter, 1);
+          idx = __shfl_sync(0xffffffffu, idx, 0);
+          item = idx < p.nitems ? p.order[idx] : -1;
+          if (item >= 0) {
+            const uint32_t* mrow = p.mask + (size_t)item * p.W;
+            if (p.W <= 64) {
+              // the item's selection row in two registers per lane (one
+              // coalesced load): walking its tiles then costs shuffles, not a
+              // dependent L2 round trip per mask word
+              ti.init(nullptr, p.W, p.Nk, p.chunks, p.pair);
+              ti.rb0 = lane < p.W ? __ldg(mrow + lane) : 0u;
+              ti.rb1 = 32 + lane < p.W ? __ldg(mrow + 32 + lane) : 0u;
+            } else {
+              ti.init(mrow, p.W, p.Nk, p.chunks, p.pair);
+            }
+            T = p.tiles[item];
+          }
+        }
+        if (lane == 0) {
+          bars.item_slot[slot] = item;
+          bars.item_T[slot] = T;
+          mbar_arrive(&bars.item_full[slot]);
+        }
+        if (item < 0) break;
+        const int bh = item / p.Nq, qi = item % p.Nq;
+        SOL_DCHECK(item < p.nitems && bh < p.bH && T >= 0, 1);
+        // the router's slot is released once this item's selection words are no
+        // longer read (after its last tile is issued)
+        auto release_route_slot = [&]() {
+          if (p.route_inkernel && lane == 0) mbar_arrive(&bars.rq_empty[slot]);
+        };
+        if (T == 0) {
+          release_route_slot();
+          ++n_items_done;
+          continue;
+        }
+        // Q tile into buffer q_uses % QST, once the item that used it last has
+        // issued all its S MMAs
+        const int qb = q_uses % QST;
+        const int qu = q_uses / QST;
+        if (qu > 0 && !(ok = wait_warp(&bars.q_empty[qb], (qu - 1) & 1, bars, lim, 2))) break;
+        if (leader) {
+          mbar_arrive_expect_tx(&bars.q_full[qb], TILE_BYTES);
+          uint8_t* qdst = smem + C::OFF_Q + qb * TILE_BYTES;
+  #pragma unroll
+          for (int hd = 0; hd < NSLAB; ++hd)
+            tma_load_3d(qdst + hd * SLAB, &tmQ, &bars.q_full[qb], hd * 64, qi * BM, bh, pol_q);
+        }
+        ++q_uses;
+        for (int n = 0; n < T; ++n) {
+          int kind = 0, tidx = 0, tidx2 = -1;
+          const bool has_tile = ti.next(kind, tidx, tidx2);
+          SOL_DCHECK(has_tile, 2);  // the item's tile count matches its selection
+          SOL_DCHECK(kind == 1 ? (tidx >= 0 && tidx < p.Nk && tidx2 < p.Nk && (p.pair || tidx2 < 0))
+                               : (tidx >= 0 && tidx < p.chunks),
+                     3);
+          uint32_t vm[4] = {0u, 0u, 0u, 0u};
+          if (kind == 0) {
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) vm[q] = ti.unselected(tidx * 4 + q);
+          }
+          const uint32_t gk = g + n;
+          const int ks = gk % KVST;
+          const int ku = gk / KVST;
+          // stage ks is free once the PV of its previous tile has finished
+          if (ku > 0 && !(ok = wait_warp(&bars.kv_empty[ks], (ku - 1) & 1, bars, lim, 3))) break;
+          if (leader) {
+            uint8_t* dk = smem + C::OFF_KV + (2 * ks) * TILE_BYTES;
+            uint8_t* dv = dk + TILE_BYTES;
+            TileDesc& td = bars.desc[ks];  // published by the arrive below (release)
+            td.kind = kind;
+            td.idx = tidx;
+            td.idx2 = tidx2;
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) td.vm[q] = vm[q];
+            mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
+            if (kind == 1 && p.pair) {
+              // rows [0, 64) <- key block tidx, rows [64, 128) <- key block tidx2;
+              // a tile with one block repeats it in the second half (masked out)
+              const int j2 = tidx2 >= 0 ? tidx2 : tidx;
+  #pragma unroll
+              for (int hd = 0; hd < NSLAB; ++hd) {
+                tma_load_3d(dk + hd * SLAB, &tmK, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+                tma_load_3d(dk + hd * SLAB + 64 * 128, &tmK, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+                tma_load_3d(dv + hd * SLAB, &tmV, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
+                tma_load_3d(dv + hd * SLAB + 64 * 128, &tmV, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
+              }
+            } else {
+              const CUtensorMap* mk = kind ? &tmK : &tmKb;
+              const CUtensorMap* mv = kind ? &tmV : &tmVb;
+  #pragma unroll
+              for (int hd = 0; hd < NSLAB; ++hd) {
+                tma_load_3d(dk + hd * SLAB, mk, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
+                tma_load_3d(dv + hd * SLAB, mv, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
+              }
+            }
+          }
+          gk_last = (int)gk;
+        }
+        if (!ok) break;
+        release_route_slot();
+        g += T;
+        ++n_items_done;
+        n_tiles_done += T;
+      }
+      if (!ok || bars.abort_flag) {
+        // let every copy this warp started land before the CTA exits: the last
+        // use of each ring stage is one of the ring's last issued tiles
+        for (int back = 0; back < KVST; ++back) {
+          const int gk = gk_last - back;
+          if (gk >= 0) mbar_wait(&bars.kv_full[gk % KVST], (gk / KVST) & 1, nullptr, &g_sol_status, 0, lim);
+        }
+        if (q_uses > 0) mbar_wait(&bars.q_full[0], (q_uses - 1) & 1, nullptr, &g_sol_status, 0, lim);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ================================================================ MMA issuer (whole warp, one lane issues)
+      const bool leader = elect_one();
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
+      // Shared-memory descriptors of the first ring stage and of the Q buffer;
+      // a stage or a K-step only moves the start address, the low 14-bit field
+      // (address / 16, no carry: shared memory is < 256 KB)
+      constexpr uint32_t TILE16 = TILE_BYTES >> 4;
+      const uint64_t dK0 = smem_desc_sw128(smem_u32(smem + C::OFF_KV), 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(smem_u32(smem + C::OFF_KV) + TILE_BYTES, SLAB, 1024);
+      const uint64_t dQ = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
+      static_assert(QST == 1, "one Q descriptor");
+      uint32_t g = 0;
+      int item_local = 0;  // items with T > 0 processed
+      bool issued = false;
+      bool ok = true;
+      // S_gs = Q K_gs^T into S buffer gs % 2.  The buffer last held tile gs - 2:
+      // the softmax read that S before handing over its P, and the PV that read
+      // the P was issued before this MMA by this thread, so it is done first.
+      // last: this is the item's last S; the Q buffer is released after it.
+      auto issue_s = [&](uint32_t gs, bool last, int qb) -> bool {
+        const int ks = gs % KVST;
+        if (!wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 15)) return false;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t dK = dK0 + (uint64_t)(2 * ks * TILE16);
+          const uint32_t tS = tmem + TM_S + (gs & 1) * 128;
+  #pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * SLAB + (kk & 3) * 32) >> 4;
+            mma_ss(tS, dQ + off, dK + off, IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          if (!(p.test_stall && gs == 0)) tc_commit(&bars.s_full[gs & 1]);
+          if (last) tc_commit(&bars.q_empty[qb]);  // every S MMA of this item has been issued
+        }
+        __syncwarp();
+        return true;
+      };
+      // O_h += P_h V_h for both halves of tile gp (its V arrived with its K),
+      // into the item's O bank; the bank's previous item must have been read
+      constexpr int NOB = o_banks<HD>();
+      auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+        const int pb = gp & 1;
+        const int ks = gp % KVST;
+        const int ob = item_local % NOB;
+        if (first && item_local >= NOB &&
+            !wait_warp(&bars.o_free[ob], ((item_local / NOB) - 1) & 1, bars, lim, 14))
+          return false;
+        if (!wait_warp(&bars.p_full[pb], (gp >> 1) & 1, bars, lim, 12)) return false;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t dV = dV0 + (uint64_t)(2 * ks * TILE16);
+          const uint32_t tP = tmem + TM_S + pb * 128;
+  #pragma unroll
+          for (int h = 0; h < 2; ++h) {
+  #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(tmem + TM_O + h * 128 + ob * 64, tP + h * 64 + kk * 8, dV + ((h * 8192 + kk * 2048) >> 4),
+                     IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          }
+          // frees the tile's stage and tells the softmax that O holds this PV
+          tc_commit(&bars.kv_empty[ks]);
+        }
+        __syncwarp();
+        return true;
+      };
+      for (int it = 0;; ++it) {
+        const int slot = it & 1;
+        if (!(ok = wait_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 10))) break;
+        const int item = bars.item_slot[slot];
+        const int T = bars.item_T[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
+        if (item < 0) break;
+        if (T == 0) continue;
+        const int qb = item_local % QST;
+        if (!(ok = wait_warp(&bars.q_full[qb], (item_local / QST) & 1, bars, lim, 11))) break;
+        // order: S_0, S_1, then for each tile n: PV_n, S_{n+2}
+        if (!(ok = issue_s(g, T == 1, qb))) break;
+        issued = true;
+        if (T > 1 && !(ok = issue_s(g + 1, T == 2, qb))) break;
+        for (int n = 0; n < T && ok; ++n) {
+          if (!(ok = issue_pv(g + n, n == 0))) break;
+          if (n + 2 < T && !(ok = issue_s(g + n + 2, n + 3 == T, qb))) break;
+        }
+        if (!ok) break;
+        if (leader) tc_commit(&bars.o_full[item_local % NOB]);
+        __syncwarp();
+        g += T;
+        ++item_local;
+      }
+      if (issued) {
+        // all MMAs of this CTA complete before TMEM is released
+        if (leader) tc_commit(&bars.teardown);
+        __syncwarp();
+        mbar_wait(&bars.teardown, 0, nullptr, &g_sol_status, 0, lim);
+      }
+      __syncwarp();
+    } else if (warp == ROUTER_WARP) {
+      // ================================================================ router (in-kernel routing only)
+      bool ok = true;
+      for (int it = 0; p.route_inkernel; ++it) {
+        const int slot = it & 1;
+        if (it >= 2 && !(ok = wait_warp(&bars.rq_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 5))) break;
         int idx = 0;
         if (lane == 0) idx = atomicAdd(p.work_counter, 1);
         idx = __shfl_sync(0xffffffffu, idx, 0);
-        item = idx < p.nitems ? p.order[idx] : -1;
+        const int item = idx < p.nitems ? p.order[idx] : -1;
+        int T = 0;
         if (item >= 0) {
-          const uint32_t* mrow = p.mask + (size_t)item * p.W;
-          if (p.W <= 64) {
-            // the item's selection row in two registers per lane (one
-            // coalesced load): walking its tiles then costs shuffles, not a
-            // dependent L2 round trip per mask word
-            ti.init(nullptr, p.W, p.Nk, p.chunks, p.pair);
-            ti.rb0 = lane < p.W ? __ldg(mrow + lane) : 0u;
-            ti.rb1 = 32 + lane < p.W ? __ldg(mrow + 32 + lane) : 0u;
-          } else {
-            ti.init(mrow, p.W, p.Nk, p.chunks, p.pair);
-          }
-          T = p.tiles[item];
+          uint32_t rb0, rb1;
+          T = route_row<HD>(p, item, lane, rb0, rb1);
+          if (lane < p.W) bars.rq_bits[slot][lane] = rb0;
+          if (32 + lane < p.W) bars.rq_bits[slot][32 + lane] = rb1;
         }
-      }
-      if (lane == 0) {
-        bars.item_slot[slot] = item;
-        bars.item_T[slot] = T;
-        mbar_arrive(&bars.item_full[slot]);
-      }
-      if (item < 0) break;
-      const int bh = item / p.Nq, qi = item % p.Nq;
-      SOL_DCHECK(item < p.nitems && bh < p.bH && T >= 0, 1);
-      // the router's slot is released once this item's selection words are no
-      // longer read (after its last tile is issued)
-      auto release_route_slot = [&]() {
-        if (p.route_inkernel && lane == 0) mbar_arrive(&bars.rq_empty[slot]);
-      };
-      if (T == 0) {
-        release_route_slot();
-        ++n_items_done;
-        continue;
-      }
-      // Q tile into buffer q_uses % QST, once the item that used it last has
-      // issued all its S MMAs
-      const int qb = q_uses % QST;
-      const int qu = q_uses / QST;
-      if (qu > 0 && !(ok = wait_warp(&bars.q_empty[qb], (qu - 1) & 1, bars, lim, 2))) break;
-      if (leader) {
-        mbar_arrive_expect_tx(&bars.q_full[qb], TILE_BYTES);
-        uint8_t* qdst = smem + C::OFF_Q + qb * TILE_BYTES;
-#pragma unroll
-        for (int hd = 0; hd < NSLAB; ++hd)
-          tma_load_3d(qdst + hd * SLAB, &tmQ, &bars.q_full[qb], hd * 64, qi * BM, bh, pol_q);
-      }
-      ++q_uses;
-      for (int n = 0; n < T; ++n) {
-        int kind = 0, tidx = 0, tidx2 = -1;
-        const bool has_tile = ti.next(kind, tidx, tidx2);
-        SOL_DCHECK(has_tile, 2);  // the item's tile count matches its selection
-        SOL_DCHECK(kind == 1 ? (tidx >= 0 && tidx < p.Nk && tidx2 < p.Nk && (p.pair || tidx2 < 0))
-                             : (tidx >= 0 && tidx < p.chunks),
-                   3);
-        uint32_t vm[4] = {0u, 0u, 0u, 0u};
-        if (kind == 0) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) vm[q] = ti.unselected(tidx * 4 + q);
+        __syncwarp();
+        if (lane == 0) {
+          bars.rq_item[slot] = item;
+          bars.rq_T[slot] = T;
+          mbar_arrive(&bars.rq_full[slot]);
         }
-        const uint32_t gk = g + n;
-        const int ks = gk % KVST;
-        const int ku = gk / KVST;
-        // stage ks is free once the PV of its previous tile has finished
-        if (ku > 0 && !(ok = wait_warp(&bars.kv_empty[ks], (ku - 1) & 1, bars, lim, 3))) break;
-        if (leader) {
-          uint8_t* dk = smem + C::OFF_KV + (2 * ks) * TILE_BYTES;
-          uint8_t* dv = dk + TILE_BYTES;
-          TileDesc& td = bars.desc[ks];  // published by the arrive below (release)
-          td.kind = kind;
-          td.idx = tidx;
-          td.idx2 = tidx2;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) td.vm[q] = vm[q];
-          mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
-          if (kind == 1 && p.pair) {
-            // rows [0, 64) <- key block tidx, rows [64, 128) <- key block tidx2;
-            // a tile with one block repeats it in the second half (masked out)
-            const int j2 = tidx2 >= 0 ? tidx2 : tidx;
-#pragma unroll
-            for (int hd = 0; hd < NSLAB; ++hd) {
-              tma_load_3d(dk + hd * SLAB, &tmK, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
-              tma_load_3d(dk + hd * SLAB + 64 * 128, &tmK, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
-              tma_load_3d(dv + hd * SLAB, &tmV, &bars.kv_full[ks], hd * 64, tidx * 64, bh, pol_kv);
-              tma_load_3d(dv + hd * SLAB + 64 * 128, &tmV, &bars.kv_full[ks], hd * 64, j2 * 64, bh, pol_kv);
-            }
-          } else {
-            const CUtensorMap* mk = kind ? &tmK : &tmKb;
-            const CUtensorMap* mv = kind ? &tmV : &tmVb;
-#pragma unroll
-            for (int hd = 0; hd < NSLAB; ++hd) {
-              tma_load_3d(dk + hd * SLAB, mk, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
-              tma_load_3d(dv + hd * SLAB, mv, &bars.kv_full[ks], hd * 64, tidx * BN, bh, pol_kv);
-            }
-          }
-        }
-        gk_last = (int)gk;
+        if (item < 0) break;
       }
-      if (!ok) break;
-      release_route_slot();
-      g += T;
-      ++n_items_done;
-      n_tiles_done += T;
+      (void)ok;
     }
-    if (!ok || bars.abort_flag) {
-      // let every copy this warp started land before the CTA exits: the last
-      // use of each ring stage is one of the ring's last issued tiles
-      for (int back = 0; back < KVST; ++back) {
-        const int gk = gk_last - back;
-        if (gk >= 0) mbar_wait(&bars.kv_full[gk % KVST], (gk / KVST) & 1, nullptr, &g_sol_status, 0, lim);
-      }
-      if (q_uses > 0) mbar_wait(&bars.q_full[0], (q_uses - 1) & 1, nullptr, &g_sol_status, 0, lim);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer (whole warp, one lane issues)
-    const bool leader = elect_one();
-    constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
-    constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-    // Shared-memory descriptors of the first ring stage and of the Q buffer;
-    // a stage or a K-step only moves the start address, the low 14-bit field
-    // (address / 16, no carry: shared memory is < 256 KB)
-    constexpr uint32_t TILE16 = TILE_BYTES >> 4;
-    const uint64_t dK0 = smem_desc_sw128(smem_u32(smem + C::OFF_KV), 16, 1024);
-    const uint64_t dV0 = smem_desc_sw128(smem_u32(smem + C::OFF_KV) + TILE_BYTES, SLAB, 1024);
-    const uint64_t dQ = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
-    static_assert(QST == 1, "one Q descriptor");
-    uint32_t g = 0;
-    int item_local = 0;  // items with T > 0 processed
-    bool issued = false;
+  } else if (warp >= EPI_WARP0) {
+    // ================================================================ epilogue
+    // out = (O_0 e_0 + O_1 e_1) / (l_0 e_0 + l_1 e_1), e_h = 2^(m_h - max(m_0, m_1)):
+    // the two column halves' partial softmax states of each row, merged once
+    // per item while the softmax warps go on with the next item.
+    setmaxnreg_dec<REG_EPI>();
+    constexpr int NOB = o_banks<HD>();
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    int item_local = 0;
     bool ok = true;
-    // S_gs = Q K_gs^T into S buffer gs % 2.  The buffer last held tile gs - 2:
-    // the softmax read that S before handing over its P, and the PV that read
-    // the P was issued before this MMA by this thread, so it is done first.
-    // last: this is the item's last S; the Q buffer is released after it.
-    auto issue_s = [&](uint32_t gs, bool last, int qb) -> bool {
-      const int ks = gs % KVST;
-      if (!wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 15)) return false;
-      tc_fence_after();
-      if (leader) {
-        const uint64_t dK = dK0 + (uint64_t)(2 * ks * TILE16);
-        const uint32_t tS = tmem + TM_S + (gs & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * SLAB + (kk & 3) * 32) >> 4;
-          mma_ss(tS, dQ + off, dK + off, IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-        if (!(p.test_stall && gs == 0)) tc_commit(&bars.s_full[gs & 1]);
-        if (last) tc_commit(&bars.q_empty[qb]);  // every S MMA of this item has been issued
-      }
-      __syncwarp();
-      return true;
-    };
-    // O_h += P_h V_h for both halves of tile gp (its V arrived with its K)
-    auto issue_pv = [&](uint32_t gp, bool first) -> bool {
-      const int pb = gp & 1;
-      const int ks = gp % KVST;
-      if (first && item_local > 0 && !wait_warp(&bars.o_free, (item_local - 1) & 1, bars, lim, 14)) return false;
-      if (!wait_warp(&bars.p_full[pb], (gp >> 1) & 1, bars, lim, 12)) return false;
-      tc_fence_after();
-      if (leader) {
-        const uint64_t dV = dV0 + (uint64_t)(2 * ks * TILE16);
-        const uint32_t tP = tmem + TM_S + pb * 128;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + TM_O + h * 128, tP + h * 64 + kk * 8, dV + ((h * 8192 + kk * 2048) >> 4), IDESC_PV,
-                   (first && kk == 0) ? 0u : 1u);
-        }
-        // frees the tile's stage and tells the softmax that O holds this PV
-        tc_commit(&bars.kv_empty[ks]);
-      }
-      __syncwarp();
-      return true;
-    };
     for (int it = 0;; ++it) {
       const int slot = it & 1;
-      if (!(ok = wait_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 10))) break;
+      if (!(ok = wait_warp(&bars.item_full[slot], (it >> 1) & 1, bars, lim, 40))) break;
       const int item = bars.item_slot[slot];
       const int T = bars.item_T[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (item < 0) break;
-      if (T == 0) continue;
-      const int qb = item_local % QST;
-      if (!(ok = wait_warp(&bars.q_full[qb], (item_local / QST) & 1, bars, lim, 11))) break;
-      // order: S_0, S_1, then for each tile n: PV_n, S_{n+2}
-      if (!(ok = issue_s(g, T == 1, qb))) break;
-      issued = true;
-      if (T > 1 && !(ok = issue_s(g + 1, T == 2, qb))) break;
-      for (int n = 0; n < T && ok; ++n) {
-        if (!(ok = issue_pv(g + n, n == 0))) break;
-        if (n + 2 < T && !(ok = issue_s(g + n + 2, n + 3 == T, qb))) break;
+      const int bh = item / p.Nq, qi = item % p.Nq;
+      const int n_rows = min(BM, p.L - qi * BM);
+      __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD;
+      if (T == 0) {  // keep-or-drop with nothing selected: the row is 0
+        if (row < n_rows)
+          for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+        continue;
       }
-      if (!ok) break;
-      if (leader) tc_commit(&bars.o_full);
+      const int ob = item_local % NOB;
+      if (!(ok = wait_warp(&bars.state_full, item_local & 1, bars, lim, 41))) break;
+      const float m0 = bars.xm[0][row], m1 = bars.xm[1][row];
+      const float l0 = bars.xl[0][row], l1 = bars.xl[1][row];
       __syncwarp();
-      g += T;
+      if (lane == 0) mbar_arrive(&bars.state_empty);
+      const float mm = fmaxf(m0, m1);
+      const float e0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
+      const float e1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
+      const float inv = 1.0f / (l0 * e0 + l1 * e1);
+      SOL_DCHECK(inv > 0.f && inv < INFINITY, 6);  // every block with tiles has a positive row sum
+      const float w0 = e0 * inv, w1 = e1 * inv;
+      if (!(ok = wait_warp(&bars.o_full[ob], (item_local / NOB) & 1, bars, lim, 42))) break;
+      tc_fence_after();
+      const uint32_t tO0 = tmem + lane_off + TM_O + ob * 64, tO1 = tO0 + 128;
+#pragma unroll
+      for (int q = 0; q < HD / 32; ++q) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tO0 + q * 32, a);
+        tmem_ld32(tO1 + q * 32, b);
+        tmem_wait_ld();
+        if (q == HD / 32 - 1) {  // O of this bank read: the MMA may reuse it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.o_free[ob]);
+        }
+        if (row < n_rows) {
+          // one 32-byte store per 16 columns when the output allows it
+#pragma unroll
+          for (int c = 0; c < 32; c += 16) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(a[c + 2 * e]) * w0 + __uint_as_float(b[c + 2 * e]) * w1,
+                                 __uint_as_float(a[c + 2 * e + 1]) * w0 + __uint_as_float(b[c + 2 * e + 1]) * w1);
+            if (p.out_align32) {
+              st_global_v8(orow + q * 32 + c, w);
+            } else {
+              *reinterpret_cast<uint4*>(orow + q * 32 + c) = make_uint4(w[0], w[1], w[2], w[3]);
+              *reinterpret_cast<uint4*>(orow + q * 32 + c + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+          }
+        }
+      }
       ++item_local;
     }
-    if (issued) {
-      // all MMAs of this CTA complete before TMEM is released
-      if (leader) tc_commit(&bars.teardown);
-      __syncwarp();
-      mbar_wait(&bars.teardown, 0, nullptr, &g_sol_status, 0, lim);
-    }
-    __syncwarp();
-  } else if (warp == ROUTER_WARP) {
-    // ================================================================ router (in-kernel routing only)
-    bool ok = true;
-    for (int it = 0; p.route_inkernel; ++it) {
-      const int slot = it & 1;
-      if (it >= 2 && !(ok = wait_warp(&bars.rq_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 5))) break;
-      int idx = 0;
-      if (lane == 0) idx = atomicAdd(p.work_counter, 1);
-      idx = __shfl_sync(0xffffffffu, idx, 0);
-      const int item = idx < p.nitems ? p.order[idx] : -1;
-      int T = 0;
-      if (item >= 0) {
-        uint32_t rb0, rb1;
-        T = route_row<HD>(p, item, lane, rb0, rb1);
-        if (lane < p.W) bars.rq_bits[slot][lane] = rb0;
-        if (32 + lane < p.W) bars.rq_bits[slot][32 + lane] = rb1;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        bars.rq_item[slot] = item;
-        bars.rq_T[slot] = T;
-        mbar_arrive(&bars.rq_full[slot]);
-      }
-      if (item < 0) break;
-    }
-    (void)ok;
+    // an abandoned item may leave a TMEM load in flight
+    tmem_wait_ld();
   } else {
-    // ================================================================ softmax + epilogue
-    const int half = (warp - 2) >> 2;     // column half of every S tile this warp owns
+    // ================================================================ softmax
+    setmaxnreg_inc<REG_SOFTMAX>();
+    constexpr int NOB = o_banks<HD>();
+    const int half = (warp - SOFTMAX_WARP0) >> 2;  // column half of every S tile this warp owns
     const int quad = warp & 3;            // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;     // query row within the tile
     const int col0 = half * 64;        // this half's key columns of an S tile
-    const int ocol0 = half * (HD / 2);  // this half's output columns
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tO = tmem + lane_off + TM_O + half * 128;  // this half's accumulator O_h
     const float sl2 = p.scale_log2;
     uint32_t g = 0;
     int item_local = 0;
@@ -707,14 +815,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (item < 0) break;
-      const int bh = item / p.Nq, qi = item % p.Nq;
-      const int n_rows = min(BM, p.L - qi * BM);
-      __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD + ocol0;
-      if (T == 0) {
-        if (row < n_rows)
-          for (int c = 0; c < HD / 2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-        continue;
-      }
+      if (T == 0) continue;  // the epilogue writes the zero rows
+      // this half's accumulator O_h in the item's O bank
+      const uint32_t tO = tmem + lane_off + TM_O + half * 128 + (item_local % NOB) * 64;
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < T; ++n) {
         const uint32_t gs = g + n;
@@ -803,7 +906,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float2 sl2v = make_float2(full ? sl2 : 1.f, full ? sl2 : 1.f);
         const float2 negv = make_float2(neg_m, neg_m);
         uint32_t pk[32];
-        l += exp_pack64<NPOLY>(x, sl2v, negv, pk);
+        l += exp_pack64<npoly<HD>()>(x, sl2v, negv, pk);
         // P over the first 32 columns of this half's S (already in registers).
         // The PV of tile gs - 2 read the previous P of this buffer; it was
         // issued before S of tile gs, and the s_full commit made after that S
@@ -830,61 +933,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) mbar_arrive(&bars.p_full[pb]);
       }
       if (!ok) break;
-      // epilogue: merge the two halves' softmax states, write this half's 64
-      // output columns: out = (O_0 e_0 + O_1 e_1) / (l_0 e_0 + l_1 e_1),
-      // e_h = 2^(m_h - max(m_0, m_1))
-      // (one buffer: a half may finish the next item's key loop before its
-      // partner has read this item's state, so writing waits for both reads)
-      if (item_local > 0 && !(ok = wait_warp(&bars.xread[quad], (item_local - 1) & 1, bars, lim, 27))) break;
+      // hand this half's softmax state of every row to the epilogue warps
+      // (once they have read the previous item's, which they do first)
+      if (item_local > 0 && !(ok = wait_warp(&bars.state_empty, (item_local - 1) & 1, bars, lim, 27))) break;
       bars.xm[half][row] = m_used;
       bars.xl[half][row] = l;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.xstate[quad]);
-      if (!(ok = wait_warp(&bars.o_full, item_local & 1, bars, lim, 24))) break;
-      tc_fence_after();
-      constexpr int OCH = C::OCHUNK;
-      uint32_t o0[OCH][32], o1[OCH][32];
-#pragma unroll
-      for (int q = 0; q < OCH; ++q) {
-        tmem_ld32(tmem + lane_off + TM_O + ocol0 + q * 32, o0[q]);
-        tmem_ld32(tmem + lane_off + TM_O + 128 + ocol0 + q * 32, o1[q]);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.o_free);
-      if (!(ok = wait_warp(&bars.xstate[quad], item_local & 1, bars, lim, 26))) break;
-      const float m0 = bars.xm[0][row], m1 = bars.xm[1][row];
-      const float mm = fmaxf(m0, m1);
-      const float e0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
-      const float e1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
-      const float inv = 1.0f / (bars.xl[0][row] * e0 + bars.xl[1][row] * e1);
-      SOL_DCHECK(inv > 0.f && inv < INFINITY, 6);  // every block with tiles has a positive row sum
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.xread[quad]);
-      const float w0 = e0 * inv, w1 = e1 * inv;
-      if (row < n_rows) {
-        // each thread writes its own row: one 32-byte store per 16 columns
-        // (a full sector) when the output allows it, else 16-byte stores
-#pragma unroll
-        for (int q = 0; q < OCH; ++q) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 16) {
-            uint32_t w[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(o0[q][c + 2 * e]) * w0 + __uint_as_float(o1[q][c + 2 * e]) * w1,
-                                 __uint_as_float(o0[q][c + 2 * e + 1]) * w0 +
-                                     __uint_as_float(o1[q][c + 2 * e + 1]) * w1);
-            if (p.out_align32) {
-              st_global_v8(orow + q * 32 + c, w);
-            } else {
-              *reinterpret_cast<uint4*>(orow + q * 32 + c) = make_uint4(w[0], w[1], w[2], w[3]);
-              *reinterpret_cast<uint4*>(orow + q * 32 + c + 8) = make_uint4(w[4], w[5], w[6], w[7]);
-            }
-          }
-        }
-      }
+      if (lane == 0) mbar_arrive(&bars.state_full);
       g += T;
       ++item_local;
     }
