@@ -51,21 +51,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Same test, but a thread whose phase is not complete yet is suspended until
-// it completes or about `hint_ns` pass, instead of returning at once: waiting
-// warps then take no issue slots from the warps doing the work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -83,7 +68,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    // try_wait suspends the warp until the phase completes or a short
+    // hardware time limit passes; an explicit suspend-time hint woke the
+    // waiting warps later (measured 1.5 % slower)
+    if (mbar_try_wait(bar, parity)) return true;
     if ((it & 7u) == 0u) {
       if (abort_flag && *abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
