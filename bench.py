@@ -254,10 +254,11 @@ class OracleTimer:
 
     def describe(self, n_blocks: int) -> str:
         heads = self.wl.batch * self.wl.heads
+        nq = -(-self.wl.L // self.bq)
         return (f"float64 oracle, {self.procs} processes (one head each, 1 BLAS thread): per head its pooling + "
-                f"routing and {n_blocks} of {self.wl.n_blocks} query blocks timed; the call "
-                f"({heads} heads x {self.wl.n_blocks} blocks) extrapolated as ceil({heads}/{self.procs}) x "
-                f"(route + {self.wl.n_blocks} x block)")
+                f"routing and {n_blocks} of {nq} query blocks timed; the call "
+                f"({heads} heads x {nq} blocks) extrapolated as ceil({heads}/{self.procs}) x "
+                f"(route + {nq} x block)")
 
 
 def run_reference(args, wl):
@@ -309,6 +310,8 @@ def config_of(wl, args):
                f"126 MB L2); no flush"}
     if args.block_k and args.block_k != wl.block:
         c["block_k"] = args.block_k
+    if args.block_q and args.block_q != wl.block:
+        c["block_q"] = args.block_q
     if args.diagonal_sigma:
         c["sigma"] = "diagonal estimator"
     if args.route_in_kernel:
@@ -321,12 +324,12 @@ def moments_of(args) -> str:
 
 
 def blocks_of(wl, args):
-    return (wl.block, args.block_k or wl.block)
+    return (args.block_q or wl.block, args.block_k or wl.block)
 
 
 def attention_kernel_name(wl, blk) -> str:
-    """The library runs tcgen05 for bf16, d in {64, 128}, Bq = 128, Bk in {64, 128}."""
-    tc = wl.dtype == torch.bfloat16 and wl.d in (64, 128) and blk[0] == 128 and blk[1] in (64, 128)
+    """The library runs tcgen05 for bf16, d in {64, 128}, Bq and Bk in {64, 128}."""
+    tc = wl.dtype == torch.bfloat16 and wl.d in (64, 128) and blk[0] in (64, 128) and blk[1] in (64, 128)
     return "attn_tc_kernel" if tc else "attn_simt_kernel"
 
 
@@ -334,6 +337,8 @@ def workload_key(wl, args) -> str:
     """File-name key of a workload's profile summaries: registry name, beta and
     key block size when it differs from the query block."""
     key = f"{args.workload}_beta{args.beta:g}"
+    if args.block_q and args.block_q != wl.block:
+        key += f"_bq{args.block_q}"
     if args.block_k and args.block_k != wl.block:
         key += f"_bk{args.block_k}"
     return key
@@ -519,6 +524,8 @@ def main():
     ap.add_argument("--beta", type=float, default=1.04)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block-q", type=int, default=None,
+                    help="query block size (64 or 128); default: the workload's block")
     ap.add_argument("--block-k", type=int, default=None,
                     help="key block size (default: the workload's block size, the same as the query block)")
     ap.add_argument("--route-in-kernel", action="store_true",
@@ -675,7 +682,8 @@ def main():
         "ms_per_call": ms_step,
         "selected_fraction": work["selected_fraction"],
         "near_ties": {"margin": NEAR_TIE_MARGIN, "pairs": near,
-                      "fraction_of_pairs": near / float(wl.batch * wl.heads * wl.n_blocks * -(-wl.L // blk[1]))},
+                      "fraction_of_pairs": near / float(wl.batch * wl.heads * -(-wl.L // blk[0]) *
+                                                        -(-wl.L // blk[1]))},
         "executed_tflop_per_call": work["total"] / 1e12,
         "executed_tflops": work["total"] / (ms_step * 1e-3) / 1e12,
         "pct_bf16_peak": 100.0 * work["total"] / (ms_step * 1e-3) / 1e12 / peak,

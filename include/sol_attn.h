@@ -82,9 +82,12 @@ typedef enum {
  * Eq. 9 weight of a key block is its token count); L >= 1;
  * 1 <= batch * heads <= 65535; batch * heads * L * d < 2^40;
  * ceil(L / Bk) <= 6144; beta not NaN.
- * Other values return SOL_ERR_UNSUPPORTED.  bf16 with Bq == 128 (any
- * supported d and Bk) runs the tensor-core (tcgen05/TMEM/TMA) kernel; every
- * other supported combination runs the CUDA-core kernel.
+ * Other values return SOL_ERR_UNSUPPORTED.  bf16 (any supported d, Bq and
+ * Bk) runs the tensor-core (tcgen05/TMEM/TMA) kernel; with Bq == 64 each
+ * 128-row tile holds two consecutive query blocks, which walk the union of
+ * their selections, each masking the key blocks it did not select (the
+ * results are those of one block at a time).  fp32 runs the CUDA-core
+ * kernel.
  */
 
 /*

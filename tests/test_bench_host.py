@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _args(**kw):
-    a = dict(workload="wan-720p", beta=1.04, block_k=None)
+    a = dict(workload="wan-720p", beta=1.04, block_k=None, block_q=None)
     a.update(kw)
     return argparse.Namespace(**a)
 
@@ -43,6 +43,10 @@ def test_workload_key_names_other_key_block_sizes():
     wl = I.WORKLOADS["wan-720p"]
     assert bench.workload_key(wl, _args(block_k=64)) == "wan-720p_beta1.04_bk64"
     assert bench.workload_key(wl, _args(block_k=128)) == "wan-720p_beta1.04"
+    assert bench.workload_key(wl, _args(block_q=64)) == "wan-720p_beta1.04_bq64"
+    assert bench.workload_key(wl, _args(block_q=64, block_k=64)) == "wan-720p_beta1.04_bq64_bk64"
+    assert bench.blocks_of(wl, _args(block_q=64)) == (64, 128)
+    assert bench.attention_kernel_name(wl, (64, 128)) == "attn_tc_kernel"
     assert bench.profiled_traffic("no-such-workload_beta1") is None
 
 

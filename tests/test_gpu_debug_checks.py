@@ -41,6 +41,9 @@ CASES = [  # (grid, heads, d, (Bq, Bk), beta, flags)
     ((10, 10, 10), 2, 128, (128, 128), 1.04, api.FLAG_KEEP_OR_DROP),
     ((10, 10, 10), 2, 128, (128, 64), 1.04, api.FLAG_ROUTE_IN_KERNEL | api.FLAG_DIAGONAL_SIGMA),
     ((21, 30, 52), 4, 128, (128, 128), 1.04, api.FLAG_ROUTE_IN_KERNEL),
+    ((10, 10, 10), 2, 128, (64, 128), 1.04, 0),   # 64-token query blocks, two per tile
+    ((3, 10, 31), 2, 64, (64, 64), 0.5, 0),       # L = 930: odd query-block count
+    ((10, 10, 10), 2, 128, (64, 128), 2.0, api.FLAG_KEEP_OR_DROP),
 ]
 
 

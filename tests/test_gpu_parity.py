@@ -83,9 +83,11 @@ def test_tiny_fp32_workload(beta):
 
 
 @pytest.mark.parametrize("L", [1, 5, 127, 128, 129, 300])
-@pytest.mark.parametrize("block", [128, (128, 64)])
+@pytest.mark.parametrize("block", [128, (128, 64), 64, (64, 128)])
 @pytest.mark.parametrize("beta", [-INF, 1.04, INF])
 def test_short_and_ragged_lengths(L, beta, block):
+    # with 64-token query blocks L = 1, 129 and 300 leave an odd block count:
+    # the last 128-row tile holds one query block
     Q, K, V = I.make_iid(1, 3, L, 128, seed=L, dtype=torch.bfloat16, device="cuda")
     check_case(Q, K, V, block, beta)
 
@@ -185,6 +187,16 @@ def test_image_dit(beta, name, bk):
     check_case(Q, K, V, (wl.block, bk), beta)
 
 
+@pytest.mark.parametrize("beta", [-INF, 1.04])
+@pytest.mark.parametrize("name,bk", [("image-dit", 128), ("image-dit", 64), ("image-dit-d64", 64)])
+def test_image_dit_query_blocks_of_64(beta, name, bk):
+    """The image-DiT tensors routed in 64-token query blocks (two to a
+    128-row tile on the tensor cores), every output row."""
+    wl = I.WORKLOADS[name]
+    Q, K, V = I.make_workload(wl, device="cuda")
+    check_case(Q, K, V, (64, bk), beta)
+
+
 @pytest.mark.parametrize("name,beta,bk", [("wan-480p", 1.04, 128),
                                           ("wan-720p", -INF, 128), ("wan-720p", 0.5, 128), ("wan-720p", 1.04, 128),
                                           ("wan-720p", 1.5, 128), ("wan-720p", 2.0, 128),
@@ -275,11 +287,29 @@ def check_keep_or_drop(Q, K, V, block, beta):
     return P.check_close(np.concatenate(gpu_rows), np.concatenate(ref_rows), Q.dtype, f"keep-or-drop beta={beta}")
 
 
-@pytest.mark.parametrize("block", [128, (128, 64)])
+@pytest.mark.parametrize("block", [128, (128, 64), 64, (64, 128)])
 @pytest.mark.parametrize("beta", [-INF, 0.5, 1.04, 2.0, INF])
 def test_keep_or_drop_bf16(beta, block):
     Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=8, device="cuda")  # L = 1000, ragged tail
     check_keep_or_drop(Q, K, V, block, beta)
+
+
+@pytest.mark.parametrize("block", [64, (64, 128)])
+@pytest.mark.parametrize("beta", [0.5, 1.04])
+def test_keep_or_drop_pair_with_an_empty_block(beta, block):
+    """Query block 0's rows are 0, so its pooled query is exactly 0 (in any
+    summation order), all its proxy scores are 0, sigma is 0 and Eq. 4's
+    strict comparison selects nothing: without the correction its rows are 0,
+    while block 1, which shares its 128-row tile, attends to its own
+    selection."""
+    Q, K, V = I.make_qkv((10, 10, 10), heads=2, d=128, seed=9, device="cuda")  # L = 1000
+    Q[:, :, :64] = 0
+    counts = api.stats(Q, K, beta, block)
+    assert (counts[:, :, 0] == 0).all() and (counts[:, :, 1] > 0).all()
+    err = check_keep_or_drop(Q, K, V, block, beta)
+    out = api.forward_ex(Q, K, V, beta, block, keep_or_drop=True)
+    assert (out[:, :, :64] == 0).all()
+    check_case(Q, K, V, block, beta)  # with the correction block 0 takes the pooled path
 
 
 @pytest.mark.parametrize("beta", [0.5, 1.04, INF])
@@ -374,6 +404,31 @@ def test_near_tie_counts_match_the_oracle(name, beta, margin):
     assert total > 0  # the margins above catch some pairs on these workloads
     for b in (-INF, INF):
         assert not api.near_ties(Q, K, b, wl.block, margin=margin).any()
+
+
+def test_cta_times_for_query_block_pairs():
+    """With 64-token query blocks a work item is the pair of blocks 2t and
+    2t + 1 (one 128-row tile): the items add up to heads x ceil(Nq / 2) and
+    the tiles to the union of each pair's selected blocks plus the chunks
+    that hold a block unselected by either."""
+    Q, K, V = I.make_qkv((10, 10, 10), heads=3, d=128, seed=10, device="cuda")  # L = 1000, Nq = 16
+    Q2, K2, V2 = Q[:, :, :936], K[:, :, :936], V[:, :, :936]  # L = 936: Nq = 15, the last pair is one block
+    for q, k, v in ((Q, K, V), (Q2.contiguous(), K2.contiguous(), V2.contiguous())):
+        api.forward(q, k, v, 1.04, (64, 128))
+        rows = api.cta_times()
+        counts, sel = api.stats(q, k, 1.04, (64, 128), with_mask=True)
+        sel = sel.cpu().numpy()[0]
+        H, Nq, Nk = sel.shape
+        npair = (Nq + 1) // 2
+        assert rows[:, 2].sum() == H * npair
+        tiles = 0
+        for t in range(npair):
+            rows_t = sel[:, 2 * t:2 * t + 2]
+            union = rows_t.any(axis=1)
+            unsel_any = (~rows_t).any(axis=1)
+            tiles += int(union.sum()) + int(sum(unsel_any[:, c * 128:(c + 1) * 128].any(axis=-1).sum()
+                                                for c in range(-(-Nk // 128))))
+        assert rows[:, 3].sum() == tiles
 
 
 def test_cta_times_account_for_every_item_and_tile():

@@ -113,9 +113,17 @@ cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
 }
 
 // The tensor-core kernel is built for bf16 with d in {64, 128}, query blocks
-// of 128 tokens and key blocks of 128 or 64 (two 64-token blocks share a tile).
+// of 128 or 64 tokens (two 64-token blocks share a 128-row tile) and key
+// blocks of 128 or 64 (two 64-token blocks share a tile).
 bool uses_tensor_cores(int dtype, const Geometry& g) {
-  return dtype == SOL_DTYPE_BF16 && (g.d == 128 || g.d == 64) && g.Bq == 128 && (g.Bk == 128 || g.Bk == 64);
+  return dtype == SOL_DTYPE_BF16 && (g.d == 128 || g.d == 64) && (g.Bq == 128 || g.Bq == 64) &&
+         (g.Bk == 128 || g.Bk == 64);
+}
+
+// In-kernel routing runs on the tensor-core kernel with 128-token query
+// blocks and at most 64 mask words per row.
+bool inkernel_supported(int dtype, const Geometry& g) {
+  return uses_tensor_cores(dtype, g) && g.Bq == 128 && g.W <= sol::kInKernelMaxW;
 }
 
 int pair_tiles(bool use_tc, const Geometry& g) { return use_tc && g.Bk == 64 ? 1 : 0; }
@@ -158,7 +166,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
   if (rc != SOL_OK) return rc;
   const bool use_tc = uses_tensor_cores(dtype, g);
-  if (inkernel && (!use_tc || g.W > sol::kInKernelMaxW)) return SOL_ERR_UNSUPPORTED;
+  if (inkernel && !inkernel_supported(dtype, g)) return SOL_ERR_UNSUPPORTED;
   const int op_dtype = use_tc ? 0 : 1;  // operand type of K-bar / V-bar: bf16 for tensor cores
   Scratch s;
   const size_t bytes = carve(g, use_tc ? 2 : 4, nullptr, &s);
@@ -432,8 +440,7 @@ extern "C" int sol_attn_forward_host(const void* q, const void* k, const void* v
   Geometry g;
   int rc = check_args(q, k, v, out, batch, heads, L, d, Bq, Bk, beta, &g);
   if (rc != SOL_OK) return rc;
-  if ((flags & SOL_FLAG_ROUTE_IN_KERNEL) && (!uses_tensor_cores(dtype, g) || g.W > sol::kInKernelMaxW))
-    return SOL_ERR_UNSUPPORTED;
+  if ((flags & SOL_FLAG_ROUTE_IN_KERNEL) && !inkernel_supported(dtype, g)) return SOL_ERR_UNSUPPORTED;
   const size_t slice = (size_t)L * d * (dtype == SOL_DTYPE_BF16 ? 2 : 4);  // bytes of one (batch, head) slice
   int G = slices_per_step;
   if (G == 0) {

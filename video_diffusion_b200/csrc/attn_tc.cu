@@ -1,6 +1,6 @@
 // attn_tc.cu -- the Sol-Attn attention loop on the 5th-generation tensor cores
 // (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, d = 128 or 64,
-// query blocks of 128 tokens, key blocks of 128 or 64 tokens.
+// query blocks of 128 or 64 tokens, key blocks of 128 or 64 tokens.
 //
 // What sets the pace is the softmax of each tile and the round trip it
 // waits on: P of tile n is written over S in TMEM, so S of tile n + 2 can be
@@ -24,6 +24,9 @@
 //     Only selected K/V tiles are ever loaded.  With 64-token key blocks one
 //     128-column tile holds two selected blocks, one per softmax column half
 //     (an odd count leaves the last tile's second half masked out).
+//   With 64-token query blocks one 128-row tile holds two blocks (rows 0-63
+//   and 64-127): the tile sequence is the union of their selections, and each
+//   row half masks out what its own block takes through the other path.
 //
 // Persistent CTAs, one per SM, 512 threads in four warpgroups (every
 // scheduler hosts one warp of each; the registers are rebalanced at start
@@ -103,7 +106,6 @@ constexpr int EPI_WARPS = 4;
 constexpr int REG_CONTROL = 72, REG_SOFTMAX = 176, REG_EPI = 88;
 static_assert(128 * REG_CONTROL + 256 * REG_SOFTMAX + 128 * REG_EPI <= 65536, "register split");
 constexpr uint32_t SLAB = BM * 128;  // 16 KB: 64 bf16 columns of a 128-row tile, 128-byte swizzled
-constexpr uint32_t BAR_AREA = 3072;
 
 // Shared-memory plan for head dimension HD (64 or 128).  A Q, K or V tile is
 // HD / 64 slabs; the K+V ring gets as many stages as fit (3 at d = 128, 6 at
@@ -119,6 +121,9 @@ struct Cfg {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_KV = OFF_Q + QST * TILE_BYTES;  // stage s: K at +2s tiles, V at +2s+1
   static constexpr uint32_t OFF_BAR = OFF_KV + 2 * KVST * TILE_BYTES;
+  // barriers, tile descriptors and row states: 3 KB fill the last of the
+  // 227 KB at d = 128; d = 64 leaves room for its six descriptors
+  static constexpr uint32_t BAR_AREA = HD == 128 ? 3072 : 4096;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_AREA;
 };
 static_assert(Cfg<128>::SMEM_BYTES <= 227 * 1024 && Cfg<64>::SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -155,6 +160,11 @@ __host__ __device__ constexpr bool poly_pair(int pair) {
 struct Params {
   int bH, L, Nq, Nk, W, nchunk, nitems, nk_last;
   int pair;             // 1: key blocks of 64 tokens, two per exact tile; 0: blocks of 128
+  // 1: query blocks of 64 tokens, two per 128-row tile: item t of head bh is
+  // the pair of query blocks 2t and 2t + 1 (rows [128 t, 128 t + 128)), which
+  // walks the union of their selections; 0: query blocks of 128 tokens
+  int rowpair;
+  int Ni;               // items per head: Nq, or ceil(Nq / 2) with rowpair
   float scale_log2;     // log2(e) / sqrt(d)
   float bias_full;      // log2(Bk)
   float bias_last;      // log2(nk_last)
@@ -178,11 +188,14 @@ struct Params {
 };
 
 // What the producer tells the other roles about the tile in one ring stage:
-// kind 0 = pooled chunk idx (vm: its unselected, in-range pooled keys, 4
-// words), kind 1 = exact key block idx (and idx2 for a 64-token pair, or -1).
+// kind 0 = pooled chunk idx (vm[r]: the unselected, in-range pooled keys of
+// row half r's query block, 4 words), kind 1 = exact key block idx (and idx2
+// for a 64-token pair, or -1); sel bit 2 c + r: the tile's c-th key block is
+// selected by row half r's query block.  With 128-token query blocks both row
+// halves hold the same block.
 struct TileDesc {
-  int kind, idx, idx2;
-  uint32_t vm[4];
+  int kind, idx, idx2, sel;
+  uint32_t vm[2][4];
 };
 
 template <int KVST>
@@ -209,39 +222,62 @@ struct Bars {
   float xm[2][BM];        // [column half][row] running max (log2 units)
   float xl[2][BM];        // [column half][row] row sum
 };
-static_assert(sizeof(Bars<Cfg<64>::KVST>) <= BAR_AREA && sizeof(Bars<Cfg<128>::KVST>) <= BAR_AREA,
+static_assert(sizeof(Bars<Cfg<64>::KVST>) <= Cfg<64>::BAR_AREA && sizeof(Bars<Cfg<128>::KVST>) <= Cfg<128>::BAR_AREA,
               "barrier area");
 static_assert(QST == 1, "one Q buffer");
 
 // Walks the tile sequence of one work item: pooled-key chunks holding an
 // unselected block, then the selected blocks in increasing order (one per
-// tile, or two with 64-token key blocks).  The selection words come from the
-// router's mask row in global memory, or (m == nullptr) from registers of the
-// warp: lane (w % 32) holds word w in rb0 (w < 32) or rb1.  Every lane of the
-// warp runs the same calls.
+// tile, or two with 64-token key blocks).  An item of two 64-token query
+// blocks walks the union: a key block is exact if either block selected it,
+// and a chunk is walked if it holds a block that either left unselected.
+// The selection words come from the router's mask rows in global memory, or
+// (m == nullptr) from registers of the warp: lane (w % 32) holds word w in
+// rb0 / rc0 (w < 32) or rb1 / rc1.  Every lane of the warp runs the same calls.
 struct TileIter {
-  const uint32_t* m;
-  uint32_t rb0, rb1;
+  const uint32_t* m;   // row of the (first) query block
+  const uint32_t* m2;  // row of the second query block (two == true)
+  uint32_t rb0, rb1, rc0, rc1;
+  bool two;
   int W, N, nchunk, pair;
   int chunk;     // next chunk to test
   int word;      // current mask word in the exact phase
   uint32_t bits; // remaining set bits of that word
   __device__ void init(const uint32_t* mrow, int W_, int N_, int nchunk_, int pair_) {
-    m = mrow; rb0 = rb1 = 0; W = W_; N = N_; nchunk = nchunk_; pair = pair_;
+    m = mrow; m2 = mrow; rb0 = rb1 = rc0 = rc1 = 0; two = false; W = W_; N = N_; nchunk = nchunk_; pair = pair_;
     chunk = 0; word = -1; bits = 0;
   }
-  __device__ __forceinline__ uint32_t load_word(int w) const {
-    if (m) return m[w];
-    return __shfl_sync(0xffffffffu, w < 32 ? rb0 : rb1, w & 31);
+  // mask word w of the first and the second query block (the same word for one block)
+  __device__ __forceinline__ void load_words(int w, uint32_t& a, uint32_t& b) const {
+    if (m) {
+      a = m[w];
+      b = two ? m2[w] : a;
+    } else {
+      a = __shfl_sync(0xffffffffu, w < 32 ? rb0 : rb1, w & 31);
+      b = two ? __shfl_sync(0xffffffffu, w < 32 ? rc0 : rc1, w & 31) : a;
+    }
   }
-  // unselected, in-range blocks of mask word w
-  __device__ __forceinline__ uint32_t unselected(int w) const {
-    return w < W ? (~load_word(w)) & valid_bits(w) : 0u;
+  // blocks of mask word w left unselected (and in range) by the first / the second block
+  __device__ __forceinline__ void unselected2(int w, uint32_t& ua, uint32_t& ub) const {
+    if (w >= W) { ua = ub = 0u; return; }
+    uint32_t a, b;
+    load_words(w, a, b);
+    const uint32_t v = valid_bits(w);
+    ua = ~a & v;
+    ub = ~b & v;
+  }
+  // 2 bits: key block j is selected by the first (bit 0) / the second (bit 1) block
+  __device__ __forceinline__ int sel_bits(int j) const {
+    uint32_t a, b;
+    load_words(j >> 5, a, b);
+    return (int)((a >> (j & 31)) & 1u) | (int)(((b >> (j & 31)) & 1u) << 1);
   }
   __device__ __forceinline__ int next_selected() {
     while (bits == 0) {
       if (++word >= W) return -1;
-      bits = load_word(word);
+      uint32_t a, b;
+      load_words(word, a, b);
+      bits = a | b;
     }
     const int b = __ffs(bits) - 1;
     bits &= bits - 1;
@@ -259,7 +295,11 @@ struct TileIter {
       const int c = chunk++;
       uint32_t un = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) un |= unselected(c * 4 + q);
+      for (int q = 0; q < 4; ++q) {
+        uint32_t ua, ub;
+        unselected2(c * 4 + q, ua, ub);
+        un |= ua | ub;
+      }
       if (un) { kind = 0; idx = c; return true; }
     }
     idx = next_selected();
@@ -479,9 +519,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           int idx = 0;
           if (lane == 0) idx = atomicAdd(p.work_counter, 1);
           idx = __shfl_sync(0xffffffffu, idx, 0);
-          item = idx < p.nitems ? p.order[idx] : -1;
+          // pairs of 64-token query blocks are taken in their natural order
+          item = idx < p.nitems ? (p.rowpair ? idx : p.order[idx]) : -1;
           if (item >= 0) {
-            const uint32_t* mrow = p.mask + (size_t)item * p.W;
+            // mask row of the item's (first) query block, and of the second
+            // one of a pair when it exists
+            const int blk = p.rowpair ? (item / p.Ni) * p.Nq + 2 * (item % p.Ni) : item;
+            const uint32_t* mrow = p.mask + (size_t)blk * p.W;
+            const bool two = p.rowpair && 2 * (item % p.Ni) + 1 < p.Nq;
             if (p.W <= 64) {
               // the item's selection row in two registers per lane (one
               // coalesced load): walking its tiles then costs shuffles, not a
@@ -489,10 +534,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               ti.init(nullptr, p.W, p.Nk, p.chunks, p.pair);
               ti.rb0 = lane < p.W ? __ldg(mrow + lane) : 0u;
               ti.rb1 = 32 + lane < p.W ? __ldg(mrow + 32 + lane) : 0u;
+              if (two) {
+                ti.rc0 = lane < p.W ? __ldg(mrow + p.W + lane) : 0u;
+                ti.rc1 = 32 + lane < p.W ? __ldg(mrow + p.W + 32 + lane) : 0u;
+              }
             } else {
               ti.init(mrow, p.W, p.Nk, p.chunks, p.pair);
+              ti.m2 = mrow + p.W;
             }
-            T = p.tiles[item];
+            ti.two = two;
+            if (p.rowpair) {
+              // the union's tile count: one walk of a copy of the iterator
+              TileIter tc = ti;
+              int kd, i1, i2;
+              T = 0;
+              while (tc.next(kd, i1, i2)) ++T;
+            } else {
+              T = p.tiles[item];
+            }
           }
         }
         if (lane == 0) {
@@ -501,7 +560,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_arrive(&bars.item_full[slot]);
         }
         if (item < 0) break;
-        const int bh = item / p.Nq, qi = item % p.Nq;
+        const int bh = item / p.Ni, qi = item % p.Ni;  // qi: the item's 128-row tile of Q
         SOL_DCHECK(item < p.nitems && bh < p.bH && T >= 0, 1);
         // the router's slot is released once this item's selection words are no
         // longer read (after its last tile is issued)
@@ -533,10 +592,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           SOL_DCHECK(kind == 1 ? (tidx >= 0 && tidx < p.Nk && tidx2 < p.Nk && (p.pair || tidx2 < 0))
                                : (tidx >= 0 && tidx < p.chunks),
                      3);
-          uint32_t vm[4] = {0u, 0u, 0u, 0u};
+          uint32_t vm[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+          int sel = 0;
           if (kind == 0) {
   #pragma unroll
-            for (int q = 0; q < 4; ++q) vm[q] = ti.unselected(tidx * 4 + q);
+            for (int q = 0; q < 4; ++q) ti.unselected2(tidx * 4 + q, vm[0][q], vm[1][q]);
+          } else {
+            sel = !p.rowpair ? 0xf : (ti.sel_bits(tidx) | (tidx2 >= 0 ? ti.sel_bits(tidx2) << 2 : 0));
           }
           const uint32_t gk = g + n;
           const int ks = gk % KVST;
@@ -550,8 +612,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             td.kind = kind;
             td.idx = tidx;
             td.idx2 = tidx2;
+            td.sel = sel;
   #pragma unroll
-            for (int q = 0; q < 4; ++q) td.vm[q] = vm[q];
+            for (int q = 0; q < 4; ++q) {
+              td.vm[0][q] = vm[0][q];
+              td.vm[1][q] = vm[1][q];
+            }
             mbar_arrive_expect_tx(&bars.kv_full[ks], 2 * TILE_BYTES);
             if (kind == 1 && p.pair) {
               // rows [0, 64) <- key block tidx, rows [64, 128) <- key block tidx2;
@@ -738,7 +804,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (item < 0) break;
-      const int bh = item / p.Nq, qi = item % p.Nq;
+      const int bh = item / p.Ni, qi = item % p.Ni;  // the item's 128-row tile of Q and of the output
       const int n_rows = min(BM, p.L - qi * BM);
       __nv_bfloat16* orow = p.out + ((size_t)bh * p.L + (size_t)qi * BM + row) * HD;
       if (T == 0) {  // keep-or-drop with nothing selected: the row is 0
@@ -755,8 +821,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float mm = fmaxf(m0, m1);
       const float e0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
       const float e1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
-      const float inv = 1.0f / (l0 * e0 + l1 * e1);
-      SOL_DCHECK(inv > 0.f && inv < INFINITY, 6);  // every block with tiles has a positive row sum
+      // a row whose query block selected nothing without the correction
+      // (keep-or-drop; only a pair's second block can meet it here) is 0
+      const float den = l0 * e0 + l1 * e1;
+      const float inv = den > 0.f ? 1.0f / den : 0.f;
+      // every block with tiles has a positive row sum, bar that case
+      SOL_DCHECK((inv > 0.f && inv < INFINITY) || (p.rowpair && p.chunks == 0) || row >= n_rows, 6);
       const float w0 = e0 * inv, w1 = e1 * inv;
       if (!(ok = wait_warp(&bars.o_full[ob], (item_local / NOB) & 1, bars, lim, 42))) break;
       tc_fence_after();
@@ -801,6 +871,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int half = (warp - SOFTMAX_WARP0) >> 2;  // column half of every S tile this warp owns
     const int quad = warp & 3;            // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;     // query row within the tile
+    const int rh = quad >> 1;             // row half: which query block of a 64-token pair
     const int col0 = half * 64;        // this half's key columns of an S tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const float sl2 = p.scale_log2;
@@ -829,6 +900,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // the reads; the stage cannot refill before this warp hands over P
         if (!(ok = wait_warp(&bars.kv_full[ks], (gs / KVST) & 1, bars, lim, 22))) break;
         const int kind = bars.desc[ks].kind, tidx = bars.desc[ks].idx, tidx2 = bars.desc[ks].idx2;
+        const int tsel = bars.desc[ks].sel;
         SOL_DCHECK((kind == 0 && tidx < p.nchunk) || (kind == 1 && tidx < p.Nk && tidx2 < p.Nk), 4);
         tc_fence_after();
         float x[64];
@@ -846,14 +918,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
         // valid key columns of this half of an exact tile: all 64 except in
         // the last (partial) key block and in a pair tile's empty second half
+        // (none when this row half's query block did not select the block:
+        // it reaches that block through its pooled chunk)
         int nvalid = 64;
         if (kind == 1) {
           if (p.pair) {
             const int jh = half ? tidx2 : tidx;
             nvalid = jh < 0 ? 0 : (jh == p.Nk - 1 ? p.nk_last : 64);
+            if (!((tsel >> (2 * half + rh)) & 1)) nvalid = 0;
           } else {
             const int nblk = tidx == p.Nk - 1 ? p.nk_last : BN;
             nvalid = min(max(nblk - col0, 0), 64);
+            if (!((tsel >> rh) & 1)) nvalid = 0;
           }
         }
         SOL_DCHECK(nvalid >= 0 && nvalid <= 64, 5);
@@ -877,7 +953,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           } else {  // pooled chunk: unselected, in-range blocks only
             bias = p.bias_full;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) vm[q] = bars.desc[ks].vm[half * 2 + q];
+            for (int q = 0; q < 2; ++q) vm[q] = bars.desc[ks].vm[rh][half * 2 + q];
             const int jl = p.Nk - 1 - tidx * BN - col0;
             if (jl >= 0 && jl < 64 && p.bias_last != p.bias_full) {
               sc = jl;
@@ -1017,8 +1093,10 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
                            const Scratch& s, cudaStream_t st, uint64_t wait_limit_ns, int correction,
                            int route_inkernel, int test_stall) {
   CUtensorMap mQ, mK, mV, mKb, mVb;
-  // built for d in {64, 128}, query blocks of 128 tokens, key blocks of 128 or 64
-  if (g.Bq != BM || (g.Bk != BN && g.Bk != BN / 2) || (g.d != 64 && g.d != 128)) return cudaErrorInvalidValue;
+  // built for d in {64, 128}, query blocks of 128 tokens (or 64, two to a
+  // tile), key blocks of 128 or 64
+  if ((g.Bq != BM && g.Bq != BM / 2) || (g.Bk != BN && g.Bk != BN / 2) || (g.d != 64 && g.d != 128))
+    return cudaErrorInvalidValue;
   if (!make_map(&mQ, q, g.d, g.L, g.bH, BM) || !make_map(&mK, k, g.d, g.L, g.bH, g.Bk) ||
       !make_map(&mV, v, g.d, g.L, g.bH, g.Bk) || !make_map(&mKb, s.kbar_op, g.d, g.Nk, g.bH, BN) ||
       !make_map(&mVb, s.vbar_op, g.d, g.Nk, g.bH, BN))
@@ -1027,6 +1105,9 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.bH = g.bH; p.L = g.L; p.Nq = g.Nq; p.Nk = g.Nk; p.W = g.W; p.nchunk = g.nchunk; p.nitems = g.nitems;
   p.nk_last = g.nk_last;
   p.pair = g.Bk == BN / 2 ? 1 : 0;
+  p.rowpair = g.Bq == BM / 2 ? 1 : 0;
+  p.Ni = p.rowpair ? (g.Nq + 1) / 2 : g.Nq;
+  p.nitems = g.bH * p.Ni;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
   p.bias_full = (float)std::log2((double)g.Bk);
   p.bias_last = (float)std::log2((double)g.nk_last);
@@ -1039,9 +1120,9 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, void* ou
   p.out_align32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   p.scale = 1.0f / sqrtf((float)g.d);  // the router's expression, evaluated the same way
   p.qbar = s.qbar; p.kbar = s.kbar; p.tau = s.tau;
-  if (route_inkernel && (g.W > kInKernelMaxW || !s.tau)) return cudaErrorInvalidValue;
-  if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
-  return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, g.nitems, st);
+  if (route_inkernel && (g.W > kInKernelMaxW || !s.tau || p.rowpair)) return cudaErrorInvalidValue;
+  if (g.d == 128) return launch_hd<128>(mQ, mK, mV, mKb, mVb, p, p.nitems, st);
+  return launch_hd<64>(mQ, mK, mV, mKb, mVb, p, p.nitems, st);
 }
 
 int last_attn_grid() { return g_last_grid; }
