@@ -126,6 +126,10 @@ bool inkernel_supported(int dtype, const Geometry& g) {
   return uses_tensor_cores(dtype, g) && g.Bq == 128 && g.W <= sol::kInKernelMaxW;
 }
 
+// Query blocks per work item of the attention kernel: the tensor-core kernel
+// takes 64-token query blocks two at a time (one 128-row tile).
+int order_group(bool use_tc, const Geometry& g) { return use_tc && g.Bq == 64 ? 2 : 1; }
+
 int pair_tiles(bool use_tc, const Geometry& g) { return use_tc && g.Bk == 64 ? 1 : 0; }
 
 int beta_mode_of(float beta) { return std::isinf(beta) ? (beta < 0 ? -1 : 1) : 0; }
@@ -185,7 +189,7 @@ int forward_impl(const void* q, const void* k, const void* v, void* out, int dty
   if ((rc = record(events, 1, st)) != SOL_OK) goto done;
   e = sol::launch_route(g, s, beta, beta_mode_of(beta), correction, sigma_mode, pair_tiles(use_tc, g), st);
   if (e != cudaSuccess) goto done;
-  e = sol::launch_order(g, s, st);
+  e = sol::launch_order(g, s, order_group(use_tc, g), st);
   if (e != cudaSuccess) goto done;
   if ((rc = record(events, 2, st)) != SOL_OK) goto done;
   if (use_tc) {
@@ -384,7 +388,7 @@ extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void
   cudaError_t e = sol::launch_pool(0, op_dtype, q, k, v, g, s, st);
   if (e == cudaSuccess)
     e = sol::launch_route(g, s, beta, beta_mode_of(beta), 1, sol::kSigmaEq5, pair_tiles(use_tc, g), st);
-  if (e == cudaSuccess) e = sol::launch_order(g, s, st);
+  if (e == cudaSuccess) e = sol::launch_order(g, s, order_group(use_tc, g), st);
   if (use_tc) {
     if (e == cudaSuccess) e = cudaMemsetAsync(s.work_counter, 0, sizeof(int32_t), st);
     if (e == cudaSuccess) e = sol::launch_attn_tc(q, k, v, out, g, s, st, wait_limit_ns(), 1, 0);

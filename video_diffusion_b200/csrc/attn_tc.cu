@@ -162,7 +162,8 @@ struct Params {
   int pair;             // 1: key blocks of 64 tokens, two per exact tile; 0: blocks of 128
   // 1: query blocks of 64 tokens, two per 128-row tile: item t of head bh is
   // the pair of query blocks 2t and 2t + 1 (rows [128 t, 128 t + 128)), which
-  // walks the union of their selections; 0: query blocks of 128 tokens
+  // walks the union of their selections (items taken heaviest first by the
+  // sum of the two blocks' tile counts); 0: query blocks of 128 tokens
   int rowpair;
   int Ni;               // items per head: Nq, or ceil(Nq / 2) with rowpair
   float scale_log2;     // log2(e) / sqrt(d)
@@ -519,8 +520,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           int idx = 0;
           if (lane == 0) idx = atomicAdd(p.work_counter, 1);
           idx = __shfl_sync(0xffffffffu, idx, 0);
-          // pairs of 64-token query blocks are taken in their natural order
-          item = idx < p.nitems ? (p.rowpair ? idx : p.order[idx]) : -1;
+          item = idx < p.nitems ? p.order[idx] : -1;
           if (item >= 0) {
             // mask row of the item's (first) query block, and of the second
             // one of a pair when it exists

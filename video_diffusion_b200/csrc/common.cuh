@@ -62,7 +62,10 @@ cudaError_t launch_pool(int in_dtype, int op_dtype, const void* q, const void* k
 // pair != 0: the attention kernel takes two selected key blocks per tile.
 cudaError_t launch_route(const Geometry& g, const Scratch& s, float beta, int beta_mode, int correction,
                          int sigma_mode, int pair, cudaStream_t st);
-cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st);
+// Heaviest-first order of the work items of each head; an item is `group`
+// consecutive query blocks (1, or 2 for the tensor-core kernel's 64-token
+// query blocks).
+cudaError_t launch_order(const Geometry& g, const Scratch& s, int group, cudaStream_t st);
 
 // Attention launches.
 // correction = 0: keep-or-drop (pooled-key tiles skipped, empty rows give 0).

@@ -410,15 +410,20 @@ __global__ void __launch_bounds__(128 * QH) route_blk_kernel(
 }
 
 // One CTA per head: bitonic sort of the head's work items by (tiles desc,
-// index asc); writes order[bh * N + rank] = bh * N + i.
-__global__ void __launch_bounds__(1024) order_kernel(const int32_t* __restrict__ tiles, int N, int P,
+// index asc); writes order[bh * NI + rank] = bh * NI + i.  A work item is G
+// consecutive query blocks (G = 1, or 2 for 64-token blocks that share a
+// 128-row tile; NI = ceil(N / G) items per head), weighed by the sum of its
+// blocks' tile counts.
+__global__ void __launch_bounds__(1024) order_kernel(const int32_t* __restrict__ tiles, int N, int G, int P,
                                                      int32_t* __restrict__ order) {
   extern __shared__ unsigned long long keys[];
   const int bh = blockIdx.x;
+  const int NI = (N + G - 1) / G;
   for (int e = threadIdx.x; e < P; e += blockDim.x) {
     unsigned long long key;
-    if (e < N) {
-      const uint32_t t = (uint32_t)tiles[(size_t)bh * N + e];
+    if (e < NI) {
+      uint32_t t = 0;
+      for (int q = G * e; q < G * e + G && q < N; ++q) t += (uint32_t)tiles[(size_t)bh * N + q];
       key = ((unsigned long long)(0x7fffffffu - t) << 32) | (uint32_t)e;
     } else {
       key = ~0ull;
@@ -442,8 +447,8 @@ __global__ void __launch_bounds__(1024) order_kernel(const int32_t* __restrict__
       __syncthreads();
     }
   }
-  for (int e = threadIdx.x; e < N; e += blockDim.x)
-    order[(size_t)bh * N + e] = bh * N + (int)(uint32_t)(keys[e] & 0xffffffffu);
+  for (int e = threadIdx.x; e < NI; e += blockDim.x)
+    order[(size_t)bh * NI + e] = bh * NI + (int)(uint32_t)(keys[e] & 0xffffffffu);
 }
 
 __global__ void identity_order_kernel(int32_t* order, int n) {
@@ -550,17 +555,18 @@ cudaError_t launch_route(const Geometry& g, const Scratch& s, float beta, int be
   return route_dispatch<64>(g, s, beta, beta_mode, correction, pair, kvar, st);
 }
 
-cudaError_t launch_order(const Geometry& g, const Scratch& s, cudaStream_t st) {
-  if (g.Nq > kOrderMaxN) {
-    identity_order_kernel<<<148, 256, 0, st>>>(s.order, g.nitems);
+cudaError_t launch_order(const Geometry& g, const Scratch& s, int group, cudaStream_t st) {
+  const int NI = (g.Nq + group - 1) / group;
+  if (NI > kOrderMaxN) {
+    identity_order_kernel<<<148, 256, 0, st>>>(s.order, g.bH * NI);
     return cudaGetLastError();
   }
   int P = 1;
-  while (P < g.Nq) P <<= 1;
+  while (P < NI) P <<= 1;
   const size_t smem = (size_t)P * sizeof(unsigned long long);
   cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  order_kernel<<<g.bH, 1024, smem, st>>>(s.tiles, g.Nq, P, s.order);
+  order_kernel<<<g.bH, 1024, smem, st>>>(s.tiles, g.Nq, group, P, s.order);
   return cudaGetLastError();
 }
 
