@@ -64,8 +64,8 @@ typedef enum {
                                      i.e. Eq. 5 with the off-diagonal covariance dropped).
                                      mu_i is unchanged. */
 #define SOL_FLAG_ROUTE_IN_KERNEL 4u /* Eq. 4 decided inside the tensor-core attention kernel
-                                     (the producer warp scores each key block from the fp32
-                                     pooled vectors with the router's arithmetic and compares
+                                     (two of its warps score each key block from the fp32
+                                     pooled vectors with the router's arithmetic and compare
                                      with the router's tau_i; Eq. 11's "proxy reuse"): no
                                      selection mask is written or read.  Same results as
                                      without the flag.  Tensor-core calls only (bf16, Bq = 128)

@@ -36,8 +36,9 @@
 //                 tile's K and V (or K-bar and V-bar) together into a 3-stage
 //                 ring (6 at d = 64)
 //   warp 1        TMEM owner and tcgen05.mma issuer (one elected lane)
-//   warp 2        in-kernel routing only: fetches the work items and decides
-//                 each one's selection ahead of the producer
+//   warps 2, 3    in-kernel routing only: fetch the work items and decide
+//                 each one's selection ahead of the producer (half the
+//                 pooled-key chunks each)
 //   warps 4..11   softmax, two column halves: half h owns the 64 keys
 //                 [64h, 64h + 64) of every tile, one query row per thread (its
 //                 warp's TMEM lane quadrant).  Each half keeps its own running
@@ -96,7 +97,7 @@ constexpr int QST = 1;  // Q buffers
 // warpgroup covers the four lane quadrants, and every scheduler (w % 4) hosts
 // one warp of each warpgroup.
 constexpr int NTHREADS = 512;
-constexpr int ROUTER_WARP = 2;  // in-kernel routing: scores the items ahead of the producer
+constexpr int ROUTER_WARP = 2;  // in-kernel routing: warps 2 and 3 score the items ahead of the producer
 constexpr int SOFTMAX_WARPS = 8;
 constexpr int SOFTMAX_WARP0 = 4;  // warps 4..11: half (w - 4) / 4, quadrant w % 4
 constexpr int EPI_WARP0 = 12;     // warps 12..15: the epilogue, quadrant w % 4
@@ -218,6 +219,8 @@ struct Bars {
   uint64_t rq_full[2], rq_empty[2];
   int rq_item[2], rq_T[2];
   uint32_t rq_bits[2][64];
+  int rr_item;            // the item the two router warps score next (router warp 0 fetches it)
+  int rr_part[2];         // router warp 1's selected-block and chunk counts
   uint32_t tmem_base;
   int abort_flag;
   float xm[2][BM];        // [column half][row] running max (log2 units)
@@ -311,27 +314,24 @@ struct TileIter {
   }
 };
 
-// Eq. 4 decided inside the kernel for query block `item`: the whole warp
-// forms s_ij = (Q-bar_i . K-bar_j) / sqrt(d) for every key block j, four
-// pooled keys per lane at a time, with the router's arithmetic (fp32, one
-// fused multiply-add per channel in channel order, then the scale), and keeps
-// the bits j with s_ij > tau_i as mask words: lane (w % 32) gets word w in rb0
-// (w < 32) or rb1 (W <= 64).  Q-bar_i stays in registers (lane l holds
-// channels 4l .. 4l + 3) and is broadcast with shuffles.  Returns the item's
-// tile count: pooled chunks holding an unselected block (with the correction)
-// plus the exact tiles.
+// Eq. 4 decided inside the kernel for query block `item`, over the chunks of
+// 128 pooled keys c = c0, c0 + cstep, ...: the whole warp forms
+// s_ij = (Q-bar_i . K-bar_j) / sqrt(d) for the chunk's key blocks j, four per
+// lane at a time, with the router's arithmetic (fp32, one fused multiply-add
+// per channel in channel order, then the scale), and writes the bits j with
+// s_ij > tau_i as the chunk's mask words into bits (shared memory).  Q-bar_i
+// is read with broadcast loads (every lane the same address).  Adds to cnt the
+// selected blocks and to used the chunks holding an unselected block.
 template <int HD>
-__device__ int route_row(const Params& p, int item, int lane, uint32_t& rb0, uint32_t& rb1) {
+__device__ void route_part(const Params& p, int item, int lane, int c0, int cstep, uint32_t* bits, int& cnt,
+                           int& used) {
   const int bh = item / p.Nq;
   SOL_DCHECK(p.W <= 64, 7);
-  float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (lane * 4 < HD) qv = __ldg(reinterpret_cast<const float4*>(p.qbar + (size_t)item * HD) + lane);
+  const float4* qrow = reinterpret_cast<const float4*>(p.qbar + (size_t)item * HD);
   const float tau = __ldg(p.tau + item);
   const float* kb = p.kbar + (size_t)bh * p.Nk * HD;
-  rb0 = rb1 = 0u;
-  int cnt = 0, used = 0;
   const int nch = (p.Nk + 127) >> 7;
-  for (int c = 0; c < nch; ++c) {
+  for (int c = c0; c < nch; c += cstep) {
     float acc[4];
     const float* kr[4];
 #pragma unroll
@@ -342,15 +342,14 @@ __device__ int route_row(const Params& p, int item, int lane, uint32_t& rb0, uin
     }
 #pragma unroll 4
     for (int cc = 0; cc < HD; cc += 4) {
-      const float qx = __shfl_sync(0xffffffffu, qv.x, cc >> 2), qy = __shfl_sync(0xffffffffu, qv.y, cc >> 2);
-      const float qz = __shfl_sync(0xffffffffu, qv.z, cc >> 2), qw = __shfl_sync(0xffffffffu, qv.w, cc >> 2);
+      const float4 q4 = __ldg(qrow + (cc >> 2));
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const float4 k4 = __ldg(reinterpret_cast<const float4*>(kr[r] + cc));
-        acc[r] = fmaf(qx, k4.x, acc[r]);
-        acc[r] = fmaf(qy, k4.y, acc[r]);
-        acc[r] = fmaf(qz, k4.z, acc[r]);
-        acc[r] = fmaf(qw, k4.w, acc[r]);
+        acc[r] = fmaf(q4.x, k4.x, acc[r]);
+        acc[r] = fmaf(q4.y, k4.y, acc[r]);
+        acc[r] = fmaf(q4.z, k4.z, acc[r]);
+        acc[r] = fmaf(q4.w, k4.w, acc[r]);
       }
     }
     bool any_unselected = false;
@@ -360,10 +359,7 @@ __device__ int route_row(const Params& p, int item, int lane, uint32_t& rb0, uin
       const bool bit = (32 * w + lane < p.Nk) && (acc[r] * p.scale > tau);
       const uint32_t word = __ballot_sync(0xffffffffu, bit);
       if (w < p.W) {
-        if (lane == (w & 31)) {
-          if (w < 32) rb0 = word;
-          else rb1 = word;
-        }
+        if (lane == 0) bits[w] = word;
         cnt += __popc(word);
         const int nb = p.Nk - w * 32;
         const uint32_t valid = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
@@ -372,8 +368,10 @@ __device__ int route_row(const Params& p, int item, int lane, uint32_t& rb0, uin
     }
     used += any_unselected ? 1 : 0;
   }
-  return (p.chunks ? used : 0) + (p.pair ? (cnt + 1) >> 1 : cnt);
 }
+
+// Named barrier of the two router warps (warps 2 and 3, 64 threads).
+__device__ __forceinline__ void router_bar() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
 
 // All 32 lanes wait; the outcome is made warp-uniform so that warp-wide
 // instructions that follow are never reached by part of a warp.
@@ -757,32 +755,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_wait(&bars.teardown, 0, nullptr, &g_sol_status, 0, lim);
       }
       __syncwarp();
-    } else if (warp == ROUTER_WARP) {
+    } else if (warp == ROUTER_WARP || warp == ROUTER_WARP + 1) {
       // ================================================================ router (in-kernel routing only)
-      bool ok = true;
+      // Two warps on two schedulers share each item's scoring (even and
+      // odd chunks of pooled keys), so neither scheduler's softmax warps
+      // lose the whole of it.  Router warp 0 fetches the item and hands the
+      // result to the producer; the warps meet at two named barriers per
+      // item, which both always reach (a failed wait ends the loop through
+      // item = -1, not by leaving early).
+      const int rw = warp - ROUTER_WARP;
       for (int it = 0; p.route_inkernel; ++it) {
         const int slot = it & 1;
-        if (it >= 2 && !(ok = wait_warp(&bars.rq_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 5))) break;
-        int idx = 0;
-        if (lane == 0) idx = atomicAdd(p.work_counter, 1);
-        idx = __shfl_sync(0xffffffffu, idx, 0);
-        const int item = idx < p.nitems ? p.order[idx] : -1;
-        int T = 0;
-        if (item >= 0) {
-          uint32_t rb0, rb1;
-          T = route_row<HD>(p, item, lane, rb0, rb1);
-          if (lane < p.W) bars.rq_bits[slot][lane] = rb0;
-          if (32 + lane < p.W) bars.rq_bits[slot][32 + lane] = rb1;
+        if (rw == 0) {
+          bool ok = true;
+          if (it >= 2) ok = wait_warp(&bars.rq_empty[slot], ((it >> 1) + 1) & 1, bars, lim, 5);
+          int idx = 0;
+          if (lane == 0 && ok) idx = atomicAdd(p.work_counter, 1);
+          idx = __shfl_sync(0xffffffffu, idx, 0);
+          if (lane == 0) bars.rr_item = ok && idx < p.nitems ? p.order[idx] : -1;
         }
-        __syncwarp();
-        if (lane == 0) {
-          bars.rq_item[slot] = item;
-          bars.rq_T[slot] = T;
-          mbar_arrive(&bars.rq_full[slot]);
+        router_bar();
+        const int item = bars.rr_item;
+        int cnt = 0, used = 0;
+        if (item >= 0) route_part<HD>(p, item, lane, rw, 2, bars.rq_bits[slot], cnt, used);
+        if (rw == 1 && lane == 0) {
+          bars.rr_part[0] = cnt;
+          bars.rr_part[1] = used;
+        }
+        router_bar();
+        if (rw == 0) {
+          cnt += bars.rr_part[0];
+          used += bars.rr_part[1];
+          const int T = item < 0 ? 0 : (p.chunks ? used : 0) + (p.pair ? (cnt + 1) >> 1 : cnt);
+          __syncwarp();
+          if (lane == 0) {
+            bars.rq_item[slot] = item;
+            bars.rq_T[slot] = T;
+            mbar_arrive(&bars.rq_full[slot]);
+          }
         }
         if (item < 0) break;
       }
-      (void)ok;
     }
   } else if (warp >= EPI_WARP0) {
     // ================================================================ epilogue
