@@ -541,7 +541,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               ti.m2 = mrow + p.W;
             }
             ti.two = two;
-            if (p.rowpair) {
+            if (p.rowpair && p.W <= 64) {
+              // the union's tile count from the rows in registers: selected
+              // blocks of either query block, and the chunks (4 words each)
+              // holding a block that either left unselected
+              const uint32_t a0 = ti.rb0, a1 = ti.rb1;
+              const uint32_t b0 = two ? ti.rc0 : a0, b1 = two ? ti.rc1 : a1;
+              const int cnt = __reduce_add_sync(0xffffffffu, __popc(a0 | b0) + __popc(a1 | b1));
+              const uint32_t f0 = __ballot_sync(0xffffffffu, lane < p.W && (~(a0 & b0) & ti.valid_bits(lane)) != 0u);
+              const uint32_t f1 =
+                  __ballot_sync(0xffffffffu, 32 + lane < p.W && (~(a1 & b1) & ti.valid_bits(32 + lane)) != 0u);
+              int used = 0;
+              for (int c = 0; c < p.chunks; ++c) used += (((c < 8 ? f0 >> (4 * c) : f1 >> (4 * (c - 8))) & 0xfu) != 0u);
+              T = used + (p.pair ? (cnt + 1) >> 1 : cnt);
+            } else if (p.rowpair) {
               // the union's tile count: one walk of a copy of the iterator
               TileIter tc = ti;
               int kd, i1, i2;
