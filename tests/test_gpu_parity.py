@@ -252,6 +252,32 @@ def test_many_key_blocks(grid, d, bk, diagonal):
     check_case(Q, K, V, (128, bk), 1.04, sample_k=4, seed=3, diagonal=diagonal)
 
 
+def test_query_block_pairs_with_long_selection_rows():
+    """64-token query and key blocks with more than 64 mask words per row
+    (L = 192000: Nq = Nk = 3000, 94 words): the producer counts a pair's
+    union tiles by walking the rows from global memory instead of from
+    registers; outputs match the oracle and the per-CTA record adds up to the
+    union tiles."""
+    Q, K, V = I.make_qkv((15, 100, 128), heads=1, d=128, seed=43, device="cuda")
+    check_case(Q, K, V, (64, 64), 1.04, sample_k=4, seed=5)
+    api.forward(Q, K, V, 1.04, (64, 64))
+    rows = api.cta_times()
+    counts, sel = api.stats(Q, K, 1.04, (64, 64), with_mask=True)
+    sel = sel.cpu().numpy()[0, 0]
+    Nq, Nk = sel.shape
+    assert -(-Nk // 32) > 64
+    a, b = sel[0::2], sel[1::2]
+    if b.shape[0] < a.shape[0]:
+        b = np.concatenate([b, a[-1:]])  # a lone last block pairs with itself
+    union = a | b
+    unsel = ~(a & b)
+    chunks = -(-Nk // 128)
+    unsel_chunks = sum(int(unsel[:, c * 128:(c + 1) * 128].any(axis=-1).sum()) for c in range(chunks))
+    exact_tiles = int(((union.sum(axis=-1) + 1) // 2).sum())  # two 64-token key blocks per tile
+    assert rows[:, 2].sum() == a.shape[0]
+    assert rows[:, 3].sum() == exact_tiles + unsel_chunks
+
+
 @pytest.mark.parametrize("d", [128, 64])
 def test_largest_supported_key_block_count(d):
     """Nk = 6144, the most pooled keys per head the library accepts (L = 393216
